@@ -1,0 +1,187 @@
+"""Float64 CPU oracle for Mixture-of-Depths Attention (MoDA).
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+baseline / reference arm of ``bench.py`` may import or call this module. The
+product path (``depth_kv_attention_b200``) never touches it, and this module
+imports nothing from the product.
+
+What it computes (the "read" step of MoDA):
+
+  For every batch b, query head h, position t, with kv-head g = h // G
+  (G = Hq / Hkv, contiguous head groups):
+
+    s_j   = scale * <q[b,t,h], k[b,j,g]>          j = 0..t      (causal)
+    s'_i  = scale * <q[b,t,h], kd[b,t,i,g]>       i = 0..Ld-1   (same token)
+    one softmax over the concatenation [s || s']
+    out[b,t,h] = sum_j p_j v[b,j,g] + sum_i p'_i vd[b,t,i,g]
+    lse[b,h,t] = log( sum_j e^{s_j} + sum_i e^{s'_i} )     (natural log)
+
+Sources:
+  * "动态混合深度注意力机制MoDA技术解析" (mhpn.cn blog), §1.2: the MoDA attention
+    formula, a single softmax over the concatenated logits of the current
+    layer's keys and the keys of the preceding layers, divided by sqrt(d),
+    times the concatenated values.
+  * same page, §2.2 "dual mask": the sequence mask lets a token see itself and
+    earlier positions; the depth mask lets a query see only the depth entries
+    of its own position.
+  * "Mixture-of-Depths Attention" (gist.science, German technical summary),
+    §2 "Methodik", Read-Step and Unified Softmax: a query at position t reads
+    the depth keys/values of the same position t from layers 0..l-1, and both
+    score sets are normalised by one softmax.
+  * "Mixture-of-Depths Attention" (gist.science, French technical summary),
+    §2 "Méthodologie", Opération: one unified softmax over sequence and depth.
+
+Readings where the pages are silent (each also listed in the design doc):
+  * the depth logits take the same ``scale`` as the sequence logits (the §1.2
+    formula divides the whole concatenation by sqrt(d));
+  * GQA maps query head h to kv-head h // G;
+  * ``lse`` is the natural log of the softmax denominator of the scaled logits;
+  * the backward pass is the derivative of the forward above (the pages give
+    none); it is pinned by central finite differences in the tests.
+
+All arithmetic is float64. Inputs may be numpy arrays or torch tensors of any
+float dtype; they are upcast exactly (bf16 -> float32 -> float64 is exact).
+The concatenated logit row is materialised explicitly, in blocks of at most
+``row_block`` query rows per (b, h), and normalised with a two-pass softmax.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = ["to_f64", "forward", "forward_rows", "backward"]
+
+
+def to_f64(x) -> np.ndarray:
+    """Exact upcast of a numpy array or torch tensor to a float64 array."""
+    if hasattr(x, "detach"):  # torch tensor, without importing torch here
+        x = x.detach().to("cpu")
+        if str(x.dtype) in ("torch.bfloat16", "torch.float16"):
+            x = x.float()
+        x = x.numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def _dims(q, k, kd):
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    Ld = kd.shape[2]
+    return B, T, Hq, Hkv, Hq // Hkv, d, Ld
+
+
+def _concat_logits(qr, kseq, kdep, scale, ts):
+    """Concatenated logit rows [sequence || depth] for query rows ``qr``.
+
+    qr   [R, d]   query vectors of positions ``ts`` (one head)
+    kseq [J, d]   sequence keys 0..J-1 of the head's kv-head
+    kdep [R, Ld, d] depth keys of the SAME positions ``ts``
+    Returns s [R, J + Ld] with -inf where the causal mask hides a key.
+    """
+    s_seq = scale * (qr @ kseq.T)                            # [R, J]
+    j = np.arange(kseq.shape[0])
+    s_seq = np.where(j[None, :] <= np.asarray(ts)[:, None], s_seq, -np.inf)
+    s_dep = scale * np.einsum("rc,ric->ri", qr, kdep)        # [R, Ld]
+    return np.concatenate([s_seq, s_dep], axis=1)
+
+
+def _softmax_rows(s):
+    """Two-pass softmax of each row; returns (p, lse)."""
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    z = np.sum(e, axis=1, keepdims=True)
+    return e / z, (m + np.log(z))[:, 0]
+
+
+def forward(q, k, v, kd, vd, scale: float, row_block: int = 256):
+    """Full MoDA forward. Returns (out [B,T,Hq,d], lse [B,Hq,T]) in float64."""
+    q, k, v, kd, vd = (to_f64(x) for x in (q, k, v, kd, vd))
+    B, T, Hq, Hkv, G, d, Ld = _dims(q, k, kd)
+    out = np.empty((B, T, Hq, d))
+    lse = np.empty((B, Hq, T))
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            for t0 in range(0, T, row_block):
+                t1 = min(T, t0 + row_block)
+                ts = np.arange(t0, t1)
+                s = _concat_logits(q[b, t0:t1, h], k[b, :t1, g],
+                                   kd[b, t0:t1, :, g], scale, ts)
+                p, l = _softmax_rows(s)
+                vals = p[:, :t1] @ v[b, :t1, g]
+                vals += np.einsum("ri,ric->rc", p[:, t1:], vd[b, t0:t1, :, g])
+                out[b, t0:t1, h] = vals
+                lse[b, h, t0:t1] = l
+    return out, lse
+
+
+def forward_rows(q, k, v, kd, vd, scale: float, b: int, h: int, ts):
+    """MoDA forward for selected positions ``ts`` of one (b, h).
+
+    Same definition as ``forward``; used to check long sequences on sampled
+    rows. Returns (out [R, d], lse [R]).
+    """
+    ts = np.asarray(sorted(int(t) for t in ts))
+    idx = [int(t) for t in ts]
+    Hq, Hkv = q.shape[2], k.shape[2]
+    g = h // (Hq // Hkv)
+    jmax = int(ts.max()) + 1
+    qr = to_f64(q[b][idx])[:, h]
+    kseq = to_f64(k[b, :jmax, g])
+    vseq = to_f64(v[b, :jmax, g])
+    kdep = to_f64(kd[b][idx])[:, :, g]
+    vdep = to_f64(vd[b][idx])[:, :, g]
+    s = _concat_logits(qr, kseq, kdep, scale, ts)
+    p, l = _softmax_rows(s)
+    vals = p[:, :jmax] @ vseq + np.einsum("ri,ric->rc", p[:, jmax:], vdep)
+    return vals, l
+
+
+def backward(q, k, v, kd, vd, dout, scale: float, row_block: int = 256):
+    """Gradients of the MoDA forward for upstream gradient ``dout``.
+
+    The pages describe no backward pass; this is the derivative of the
+    forward definition above (softmax Jacobian), written per row block:
+
+      P   = exp(s - lse)                  (the forward's probabilities)
+      D   = <dout, out>                   per row
+      dP  = [dout . v_j  ||  dout . vd_i]
+      dS  = P * (dP - D)
+      dq  = scale * (sum_j dS_j k_j + sum_i dS'_i kd_i)
+      dk_j  += scale * dS_j q      dv_j  += P_j dout      (summed over rows)
+      dkd_i += scale * dS'_i q     dvd_i += P'_i dout     (same position)
+
+    Returns (dq, dk, dv, dkd, dvd, out, lse), all float64.
+    """
+    q, k, v, kd, vd, dout = (to_f64(x) for x in (q, k, v, kd, vd, dout))
+    B, T, Hq, Hkv, G, d, Ld = _dims(q, k, kd)
+    out, lse = forward(q, k, v, kd, vd, scale, row_block)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    dkd = np.zeros_like(kd)
+    dvd = np.zeros_like(vd)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            for t0 in range(0, T, row_block):
+                t1 = min(T, t0 + row_block)
+                ts = np.arange(t0, t1)
+                qr = q[b, t0:t1, h]
+                dor = dout[b, t0:t1, h]
+                s = _concat_logits(qr, k[b, :t1, g], kd[b, t0:t1, :, g], scale, ts)
+                P = np.exp(s - lse[b, h, t0:t1][:, None])
+                D = np.sum(dor * out[b, t0:t1, h], axis=1)
+                dP_seq = dor @ v[b, :t1, g].T
+                dP_dep = np.einsum("rc,ric->ri", dor, vd[b, t0:t1, :, g])
+                dP = np.concatenate([dP_seq, dP_dep], axis=1)
+                dS = P * (dP - D[:, None])
+                dS_seq, dS_dep = dS[:, :t1], dS[:, t1:]
+                P_seq, P_dep = P[:, :t1], P[:, t1:]
+                dq[b, t0:t1, h] = scale * (dS_seq @ k[b, :t1, g]
+                                           + np.einsum("ri,ric->rc", dS_dep, kd[b, t0:t1, :, g]))
+                dk[b, :t1, g] += scale * (dS_seq.T @ qr)
+                dv[b, :t1, g] += P_seq.T @ dor
+                dkd[b, t0:t1, :, g] += scale * dS_dep[:, :, None] * qr[:, None, :]
+                dvd[b, t0:t1, :, g] += P_dep[:, :, None] * dor[:, None, :]
+    return dq, dk, dv, dkd, dvd, out, lse
