@@ -1,0 +1,234 @@
+"""Python binding of the MoDA C ABI (``libmoda.so``, header ``include/moda.h``).
+
+Argument marshalling only: every function forwards torch CUDA tensors' device
+pointers and the current CUDA stream to the C entry point of the same name.
+All arithmetic runs in the library's CUDA kernels. There is no CPU fallback:
+importing this package fails if the library has not been built
+(``python -m depth_kv_attention_b200.build``).
+
+Layouts (contiguous): q/out/dout [B,T,Hq,d]; k/v [B,T,Hkv,d];
+kd/vd [B,T,Ld,Hkv,d]; lse [B,Hq,T] fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "MODA_OK", "ModaError", "lib", "LIB_PATH", "moda_abi_version", "moda_status_string",
+    "moda_fwd", "moda_bwd", "moda_bwd_workspace_bytes", "moda_pack_depth",
+    "moda_pack_depth_bytes", "moda_fwd_packed", "moda_device_status",
+    "moda_debug_set_wait_limit", "moda_fwd_from_host",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoda.so")
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m depth_kv_attention_b200.build` "
+        "(the MoDA path has no CPU fallback)")
+lib = ctypes.CDLL(LIB_PATH)
+
+MODA_OK = 0
+_DTYPE = {torch.bfloat16: 0, torch.float32: 1}
+_IMPL = {"auto": 0, "simt": 1, "tc": 2}
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+
+def _sig(name, res, args):
+    fn = getattr(lib, name)
+    fn.restype = res
+    fn.argtypes = args
+    return fn
+
+
+_DIMS = [_i] * 6  # B, T, Hq, Hkv, d, Ld
+_c_abi_version = _sig("moda_abi_version", _i, [])
+_c_status_string = _sig("moda_status_string", ctypes.c_char_p, [_i])
+_c_fwd_ex = _sig("moda_fwd_ex", _i, [_vp] * 5 + _DIMS + [_i, _f, _vp, _vp, _vp, _i])
+_c_fwd = _sig("moda_fwd", _i, [_vp] * 5 + _DIMS + [_i, _f, _vp, _vp, _vp])
+_c_bwd_ws = _sig("moda_bwd_workspace_bytes", _sz, _DIMS + [_i])
+_c_bwd_ex = _sig("moda_bwd_ex", _i, [_vp] * 8 + _DIMS + [_i, _f] + [_vp] * 5 + [_vp, _sz, _vp, _i])
+_c_bwd = _sig("moda_bwd", _i, [_vp] * 8 + _DIMS + [_i, _f] + [_vp] * 5 + [_vp, _sz, _vp])
+_c_pack_bytes = _sig("moda_pack_depth_bytes", _sz, [_i] * 5 + [_i])
+_c_pack = _sig("moda_pack_depth", _i, [_vp, _vp] + [_i] * 5 + [_i, _vp, _vp])
+_c_fwd_packed = _sig("moda_fwd_packed", _i, [_vp] * 4 + _DIMS + [_i, _f, _vp, _vp, _vp])
+_c_dev_status = _sig("moda_device_status", _i, [_vp])
+_c_wait_limit = _sig("moda_debug_set_wait_limit", _i, [ctypes.c_uint32])
+
+
+class ModaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {moda_status_string(code)} ({code})")
+
+
+def moda_abi_version() -> int:
+    return _c_abi_version()
+
+
+def moda_status_string(code: int) -> str:
+    return _c_status_string(code).decode()
+
+
+def _check(code: int, where: str) -> None:
+    if code != MODA_OK:
+        raise ModaError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dims(q, k, kd):
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    Ld = 0 if kd is None else kd.shape[2]
+    return B, T, Hq, Hkv, d, Ld
+
+
+def _check_tensors(*ts):
+    dev = None
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("MoDA tensors must be CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("MoDA tensors must be contiguous")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("MoDA tensors must be on one device")
+
+
+def moda_fwd(q, k, v, kd=None, vd=None, scale: float | None = None, out=None, lse=None,
+             impl: str = "auto", stream=None):
+    """MoDA forward (``moda_fwd_ex``). Returns (out, lse)."""
+    if kd is not None and kd.shape[2] == 0:
+        kd = vd = None
+    _check_tensors(q, k, v, kd, vd, out, lse)
+    B, T, Hq, Hkv, d, Ld = _dims(q, k, kd)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
+    with torch.cuda.device(q.device):
+        _check(_c_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(kd), _ptr(vd), B, T, Hq, Hkv, d, Ld,
+                         _DTYPE[q.dtype], scale, _ptr(out), _ptr(lse), _stream(stream), _IMPL[impl]),
+               "moda_fwd")
+    return out, lse
+
+
+def moda_bwd_workspace_bytes(B, T, Hq, Hkv, d, Ld, dtype) -> int:
+    return _c_bwd_ws(B, T, Hq, Hkv, d, Ld, _DTYPE[dtype])
+
+
+def moda_bwd(q, k, v, kd, vd, out, lse, dout, scale: float | None = None, grads=None,
+             workspace=None, impl: str = "auto", stream=None):
+    """MoDA backward (``moda_bwd_ex``). Returns (dq, dk, dv, dkd, dvd)."""
+    if kd is not None and kd.shape[2] == 0:
+        kd = vd = None
+    _check_tensors(q, k, v, kd, vd, out, lse, dout)
+    B, T, Hq, Hkv, d, Ld = _dims(q, k, kd)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                 None if kd is None else torch.empty_like(kd),
+                 None if vd is None else torch.empty_like(vd))
+    dq, dk, dv, dkd, dvd = grads
+    need = moda_bwd_workspace_bytes(B, T, Hq, Hkv, d, Ld, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    with torch.cuda.device(q.device):
+        _check(_c_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(kd), _ptr(vd), _ptr(out), _ptr(lse),
+                         _ptr(dout), B, T, Hq, Hkv, d, Ld, _DTYPE[q.dtype], scale, _ptr(dq),
+                         _ptr(dk), _ptr(dv), _ptr(dkd), _ptr(dvd), _ptr(workspace),
+                         workspace.numel(), _stream(stream), _IMPL[impl]), "moda_bwd")
+    return dq, dk, dv, dkd, dvd
+
+
+def moda_pack_depth_bytes(B, T, Hkv, d, Ld, dtype) -> int:
+    return _c_pack_bytes(B, T, Hkv, d, Ld, _DTYPE[dtype])
+
+
+def moda_pack_depth(kd, vd, packed=None, stream=None):
+    """Repack kd, vd [B,T,Ld,Hkv,d] into [2,B,Hkv,T*Ld,d] (``moda_pack_depth``)."""
+    _check_tensors(kd, vd, packed)
+    B, T, Ld, Hkv, d = kd.shape
+    n = moda_pack_depth_bytes(B, T, Hkv, d, Ld, kd.dtype)
+    if packed is None:
+        packed = torch.empty(n // kd.element_size(), device=kd.device, dtype=kd.dtype)
+    with torch.cuda.device(kd.device):
+        _check(_c_pack(_ptr(kd), _ptr(vd), B, T, Hkv, d, Ld, _DTYPE[kd.dtype], _ptr(packed),
+                       _stream(stream)), "moda_pack_depth")
+    return packed
+
+
+def moda_fwd_packed(q, k, v, packed, Ld: int, scale: float | None = None, out=None, lse=None,
+                    stream=None):
+    """MoDA forward reading depth from ``moda_pack_depth``'s layout."""
+    _check_tensors(q, k, v, packed, out, lse)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
+    with torch.cuda.device(q.device):
+        _check(_c_fwd_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(packed) if Ld else None, B, T, Hq,
+                             Hkv, d, Ld, _DTYPE[q.dtype], scale, _ptr(out), _ptr(lse),
+                             _stream(stream)), "moda_fwd_packed")
+    return out, lse
+
+
+def moda_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return _c_dev_status(_stream(stream))
+
+
+def moda_debug_set_wait_limit(spins: int) -> None:
+    _check(_c_wait_limit(spins), "moda_debug_set_wait_limit")
+
+
+def moda_fwd_from_host(q, k, v, kd=None, vd=None, scale: float | None = None, device="cuda",
+                       out_host=None, lse_host=None, dev_bufs=None, impl: str = "auto"):
+    """End-to-end forward from HOST tensors: copy inputs host->device on the
+    current stream, run ``moda_fwd``, copy out and lse back to host buffers.
+
+    ``out_host`` / ``lse_host`` (pinned CPU tensors) are filled in place when
+    given. ``dev_bufs`` may hold pre-allocated device buffers
+    (q,k,v,kd,vd,out,lse) to keep allocation out of a timed loop.
+    Returns (out_host, lse_host) after the stream has finished.
+    """
+    B, T, Hq, d = q.shape
+    if dev_bufs is None:
+        dev_bufs = {n: (None if t is None else torch.empty(t.shape, dtype=t.dtype, device=device))
+                    for n, t in dict(q=q, k=k, v=v, kd=kd, vd=vd).items()}
+        dev_bufs["out"] = torch.empty(q.shape, dtype=q.dtype, device=device)
+        dev_bufs["lse"] = torch.empty((B, Hq, T), dtype=torch.float32, device=device)
+    for n, t in dict(q=q, k=k, v=v, kd=kd, vd=vd).items():
+        if t is not None:
+            dev_bufs[n].copy_(t, non_blocking=True)
+    moda_fwd(dev_bufs["q"], dev_bufs["k"], dev_bufs["v"], dev_bufs["kd"], dev_bufs["vd"], scale,
+             out=dev_bufs["out"], lse=dev_bufs["lse"], impl=impl)
+    if out_host is None:
+        out_host = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    if lse_host is None:
+        lse_host = torch.empty((B, Hq, T), dtype=torch.float32, pin_memory=True)
+    out_host.copy_(dev_bufs["out"], non_blocking=True)
+    lse_host.copy_(dev_bufs["lse"], non_blocking=True)
+    torch.cuda.current_stream().synchronize()
+    return out_host, lse_host

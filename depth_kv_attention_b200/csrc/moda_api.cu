@@ -1,0 +1,241 @@
+// Host side of the C ABI declared in include/moda.h: argument validation,
+// kernel-family selection and launch. No allocation, no synchronisation
+// (except moda_device_status), no state beyond the device status word.
+#include <cstdint>
+#include <cstring>
+
+#include "moda_internal.h"
+
+namespace moda {
+
+// One word per device that a kernel sets when a bounded wait expires. It is
+// a file-scope __device__ variable, so the library itself never allocates.
+__device__ unsigned int g_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+unsigned int* g_status_ptr[kMaxDevices];
+unsigned int g_wait_limit[kMaxDevices];
+
+// Device address of the status word on the current device (resolved once per
+// device; cudaGetSymbolAddress needs the device current).
+cudaError_t status_ptr(unsigned int** p, unsigned int* wait_limit) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (!g_status_ptr[dev]) {
+        void* a = nullptr;
+        e = cudaGetSymbolAddress(&a, g_status_word);
+        if (e != cudaSuccess) return e;
+        g_status_ptr[dev] = static_cast<unsigned int*>(a);
+    }
+    *p = g_status_ptr[dev];
+    if (wait_limit) *wait_limit = g_wait_limit[dev];
+    return cudaSuccess;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moda_status check_dims(int B, int T, int Hq, int Hkv, int d, int Ld) {
+    if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || d < 1 || Ld < 0) return MODA_ERR_INVALID_VALUE;
+    if (Hq % Hkv) return MODA_ERR_INVALID_VALUE;
+    if (d > 128) return MODA_ERR_UNSUPPORTED;
+    // Row offsets are formed in 64-bit; the grid uses T and Hq in 32-bit dims.
+    if ((long long)B * T * Hq > (1LL << 40)) return MODA_ERR_UNSUPPORTED;
+    return MODA_OK;
+}
+
+moda_status fill_fwd(FwdArgs& a, const void* q, const void* k, const void* v, const void* kd,
+                     const void* vd, int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dt,
+                     float scale, void* out, float* lse, bool packed) {
+    moda_status st = check_dims(B, T, Hq, Hkv, d, Ld);
+    if (st != MODA_OK) return st;
+    if (dt != MODA_BF16 && dt != MODA_F32) return MODA_ERR_INVALID_VALUE;
+    if (!q || !k || !v || !out) return MODA_ERR_INVALID_VALUE;
+    if (Ld > 0 && (!kd || !vd)) return MODA_ERR_INVALID_VALUE;
+    if (!(scale == scale)) return MODA_ERR_INVALID_VALUE;  // NaN scale
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
+        (Ld > 0 && (!aligned16(kd) || !aligned16(vd))))
+        return MODA_ERR_MISALIGNED;
+    std::memset(&a, 0, sizeof(a));
+    a.q = q; a.k = k; a.v = v; a.kd = kd; a.vd = vd; a.out = out; a.lse = lse;
+    a.B = B; a.T = T; a.Hq = Hq; a.Hkv = Hkv; a.G = Hq / Hkv; a.d = d; a.Ld = Ld;
+    a.scale = scale;
+    a.sq = strides_q(T, Hq, d);
+    a.so = a.sq;
+    a.skv = strides_q(T, Hkv, d);
+    a.sdep = packed ? strides_depth_packed(T, Ld, Hkv, d) : strides_depth_native(T, Ld, Hkv, d);
+    a.dtype = dt;
+    return MODA_OK;
+}
+
+moda_status run_fwd(FwdArgs& a, void* stream, moda_impl impl) {
+    cudaError_t e = status_ptr(&a.status, &a.wait_limit);
+    if (e != cudaSuccess) return MODA_ERR_CUDA;
+    const bool tc_ok = fwd_tc_supported(a);
+    if (impl == MODA_IMPL_TC && !tc_ok) return MODA_ERR_UNSUPPORTED;
+    const bool use_tc = impl == MODA_IMPL_TC || (impl == MODA_IMPL_AUTO && tc_ok);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    e = use_tc ? launch_fwd_tc(a, s) : launch_fwd_simt(a, s);
+    return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
+}
+
+size_t bwd_ws_bytes(int B, int T, int Hq, int d, bool with_dq_acc) {
+    size_t rowD = (size_t)B * Hq * T * sizeof(float);
+    rowD = (rowD + 255) & ~size_t(255);
+    size_t acc = with_dq_acc ? (size_t)B * T * Hq * d * sizeof(float) : 0;
+    return rowD + acc;
+}
+
+}  // namespace
+}  // namespace moda
+
+using namespace moda;
+
+extern "C" {
+
+int moda_abi_version(void) { return MODA_ABI_VERSION; }
+
+const char* moda_status_string(moda_status s) {
+    switch (s) {
+        case MODA_OK: return "MODA_OK";
+        case MODA_ERR_INVALID_VALUE: return "MODA_ERR_INVALID_VALUE";
+        case MODA_ERR_UNSUPPORTED: return "MODA_ERR_UNSUPPORTED";
+        case MODA_ERR_MISALIGNED: return "MODA_ERR_MISALIGNED";
+        case MODA_ERR_WORKSPACE: return "MODA_ERR_WORKSPACE";
+        case MODA_ERR_LAUNCH: return "MODA_ERR_LAUNCH";
+        case MODA_ERR_DEVICE_TIMEOUT: return "MODA_ERR_DEVICE_TIMEOUT";
+        case MODA_ERR_CUDA: return "MODA_ERR_CUDA";
+    }
+    return "MODA_ERR_UNKNOWN";
+}
+
+moda_status moda_fwd_ex(const void* q, const void* k, const void* v, const void* kd, const void* vd,
+                        int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dtype, float scale,
+                        void* out, float* lse, void* stream, moda_impl impl) {
+    if (impl != MODA_IMPL_AUTO && impl != MODA_IMPL_SIMT && impl != MODA_IMPL_TC)
+        return MODA_ERR_INVALID_VALUE;
+    FwdArgs a;
+    moda_status st = fill_fwd(a, q, k, v, kd, vd, B, T, Hq, Hkv, d, Ld, dtype, scale, out, lse, false);
+    if (st != MODA_OK) return st;
+    return run_fwd(a, stream, impl);
+}
+
+moda_status moda_fwd(const void* q, const void* k, const void* v, const void* kd, const void* vd,
+                     int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dtype, float scale,
+                     void* out, float* lse, void* stream) {
+    return moda_fwd_ex(q, k, v, kd, vd, B, T, Hq, Hkv, d, Ld, dtype, scale, out, lse, stream,
+                       MODA_IMPL_AUTO);
+}
+
+size_t moda_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dtype) {
+    if (check_dims(B, T, Hq, Hkv, d, Ld) != MODA_OK) return 0;
+    if (dtype != MODA_BF16 && dtype != MODA_F32) return 0;
+    // The fp32 dQ accumulator is reserved for every bf16 shape so that the
+    // size does not depend on which kernel family a call selects.
+    return bwd_ws_bytes(B, T, Hq, d, dtype == MODA_BF16);
+}
+
+moda_status moda_bwd_ex(const void* q, const void* k, const void* v, const void* kd, const void* vd,
+                        const void* out, const float* lse, const void* dout, int B, int T, int Hq,
+                        int Hkv, int d, int Ld, moda_dtype dtype, float scale, void* dq, void* dk,
+                        void* dv, void* dkd, void* dvd, void* workspace, size_t workspace_bytes,
+                        void* stream, moda_impl impl) {
+    if (impl != MODA_IMPL_AUTO && impl != MODA_IMPL_SIMT && impl != MODA_IMPL_TC)
+        return MODA_ERR_INVALID_VALUE;
+    BwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    moda_status st = fill_fwd(a.f, q, k, v, kd, vd, B, T, Hq, Hkv, d, Ld, dtype, scale,
+                              const_cast<void*>(out), const_cast<float*>(lse), false);
+    if (st != MODA_OK) return st;
+    if (!lse || !dout || !dq || !dk || !dv) return MODA_ERR_INVALID_VALUE;
+    if (Ld > 0 && (!dkd || !dvd)) return MODA_ERR_INVALID_VALUE;
+    if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+        (Ld > 0 && (!aligned16(dkd) || !aligned16(dvd))))
+        return MODA_ERR_MISALIGNED;
+    const size_t need = moda_bwd_workspace_bytes(B, T, Hq, Hkv, d, Ld, dtype);
+    if (!workspace || workspace_bytes < need) return MODA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MODA_ERR_MISALIGNED;
+    a.dout = dout; a.dq = dq; a.dk = dk; a.dv = dv; a.dkd = dkd; a.dvd = dvd;
+    a.rowD = static_cast<float*>(workspace);
+    const size_t rowD = bwd_ws_bytes(B, T, Hq, d, false);
+    a.dq_acc = dtype == MODA_BF16 ? reinterpret_cast<float*>(static_cast<char*>(workspace) + rowD) : nullptr;
+    cudaError_t e = status_ptr(&a.f.status, &a.f.wait_limit);
+    if (e != cudaSuccess) return MODA_ERR_CUDA;
+    const bool tc_ok = bwd_tc_supported(a);
+    if (impl == MODA_IMPL_TC && !tc_ok) return MODA_ERR_UNSUPPORTED;
+    const bool use_tc = impl == MODA_IMPL_TC || (impl == MODA_IMPL_AUTO && tc_ok);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    e = use_tc ? launch_bwd_tc(a, s) : launch_bwd_simt(a, s);
+    return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
+}
+
+moda_status moda_bwd(const void* q, const void* k, const void* v, const void* kd, const void* vd,
+                     const void* out, const float* lse, const void* dout, int B, int T, int Hq,
+                     int Hkv, int d, int Ld, moda_dtype dtype, float scale, void* dq, void* dk,
+                     void* dv, void* dkd, void* dvd, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+    return moda_bwd_ex(q, k, v, kd, vd, out, lse, dout, B, T, Hq, Hkv, d, Ld, dtype, scale, dq, dk,
+                       dv, dkd, dvd, workspace, workspace_bytes, stream, MODA_IMPL_AUTO);
+}
+
+size_t moda_pack_depth_bytes(int B, int T, int Hkv, int d, int Ld, moda_dtype dtype) {
+    if (B < 1 || T < 1 || Hkv < 1 || d < 1 || d > 128 || Ld < 0) return 0;
+    if (dtype != MODA_BF16 && dtype != MODA_F32) return 0;
+    const size_t esz = dtype == MODA_F32 ? 4 : 2;
+    return 2 * (size_t)B * T * Ld * Hkv * d * esz;
+}
+
+moda_status moda_pack_depth(const void* kd, const void* vd, int B, int T, int Hkv, int d, int Ld,
+                            moda_dtype dtype, void* packed, void* stream) {
+    if (B < 1 || T < 1 || Hkv < 1 || d < 1 || Ld < 0) return MODA_ERR_INVALID_VALUE;
+    if (dtype != MODA_BF16 && dtype != MODA_F32) return MODA_ERR_INVALID_VALUE;
+    if (d > 128) return MODA_ERR_UNSUPPORTED;
+    if (Ld == 0) return MODA_OK;
+    if (!kd || !vd || !packed) return MODA_ERR_INVALID_VALUE;
+    if (!aligned16(kd) || !aligned16(vd) || !aligned16(packed)) return MODA_ERR_MISALIGNED;
+    const int esz = dtype == MODA_F32 ? 4 : 2;
+    if ((d * esz) % 16) return MODA_ERR_UNSUPPORTED;  // 16-byte vector copies
+    cudaError_t e = launch_pack_depth(kd, vd, B, T, Hkv, d, Ld, dtype, packed,
+                                      static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
+}
+
+moda_status moda_fwd_packed(const void* q, const void* k, const void* v, const void* packed_depth,
+                            int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dtype,
+                            float scale, void* out, float* lse, void* stream) {
+    const size_t half = moda_pack_depth_bytes(B, T, Hkv, d, Ld, dtype) / 2;
+    const void* kd = packed_depth;
+    const void* vd = packed_depth ? static_cast<const char*>(packed_depth) + half : nullptr;
+    FwdArgs a;
+    moda_status st = fill_fwd(a, q, k, v, kd, vd, B, T, Hq, Hkv, d, Ld, dtype, scale, out, lse, true);
+    if (st != MODA_OK) return st;
+    return run_fwd(a, stream, MODA_IMPL_AUTO);
+}
+
+moda_status moda_device_status(void* stream) {
+    unsigned int* p = nullptr;
+    if (status_ptr(&p, nullptr) != cudaSuccess) return MODA_ERR_CUDA;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MODA_ERR_CUDA;
+    unsigned int w = 0;
+    if (cudaMemcpy(&w, p, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return MODA_ERR_CUDA;
+    if (w) {
+        const unsigned int zero = 0;
+        if (cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+            return MODA_ERR_CUDA;
+        return MODA_ERR_DEVICE_TIMEOUT;
+    }
+    return MODA_OK;
+}
+
+moda_status moda_debug_set_wait_limit(uint32_t spins) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MODA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MODA_ERR_CUDA;
+    g_wait_limit[dev] = spins;
+    return MODA_OK;
+}
+
+}  // extern "C"

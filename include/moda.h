@@ -1,0 +1,198 @@
+/*
+ * moda.h — C ABI of the B200 (sm_100a) Mixture-of-Depths Attention library.
+ *
+ * The operation (the MoDA "read" step).  For batch b, query head h, position t
+ * and kv-head g = h / G (G = Hq / Hkv, contiguous head groups):
+ *
+ *     s_j  = scale * <q[b,t,h,:], k[b,j,g,:]>        for j = 0..t        (causal)
+ *     s'_i = scale * <q[b,t,h,:], kd[b,t,i,g,:]>     for i = 0..Ld-1     (same token)
+ *     p    = softmax over the concatenation [s || s']  (ONE normaliser)
+ *     out[b,t,h,:] = sum_j p_j v[b,j,g,:] + sum_i p'_i vd[b,t,i,g,:]
+ *     lse[b,h,t]   = log(sum_j e^{s_j} + sum_i e^{s'_i})     (natural log)
+ *
+ * Sources: "动态混合深度注意力机制MoDA技术解析" (mhpn.cn), §1.2 (the MoDA attention
+ * formula: one softmax over the concatenated current-layer and earlier-layer
+ * logits scaled by 1/sqrt(d)) and §2.2 (online softmax state m / acc / o, and
+ * the dual mask: causal over the sequence, same position over depth);
+ * "Mixture-of-Depths Attention" (gist.science, German technical summary),
+ * §2 "Methodik" (Read-Step, Unified Softmax, flash-compatible / chunk-aware /
+ * group-aware layouts).  Ld = 0 is plain causal GQA attention.
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor argument is a DEVICE pointer to a dense, row-major tensor in
+ *     the layout stated below, aligned to 16 bytes. The caller owns every
+ *     buffer; the library never allocates, frees or synchronises (except in
+ *     moda_device_status) and keeps no per-call state.
+ *   - Layouts:  q, out, dout, dq   [B, T, Hq, d]
+ *               k, v, dk, dv       [B, T, Hkv, d]
+ *               kd, vd, dkd, dvd   [B, T, Ld, Hkv, d]   (depth keys/values of a
+ *                                   token's earlier layers, token-contiguous)
+ *               lse                [B, Hq, T]  fp32
+ *   - dtype: MODA_BF16 (bf16 storage, fp32 accumulation) or MODA_F32 (fp32
+ *     storage and arithmetic). Outputs take the input dtype; lse and the
+ *     workspace are fp32.
+ *   - stream: a cudaStream_t cast to void*; NULL means the legacy default
+ *     stream. Every call only ENQUEUES work and returns; results are ready
+ *     when the stream reaches them.
+ *   - kd and vd may be NULL iff Ld == 0. Outputs must not alias inputs.
+ *   - Argument errors return synchronously with nothing launched. A failed
+ *     launch returns MODA_ERR_LAUNCH. A kernel whose bounded wait on an
+ *     on-chip barrier expires records MODA_ERR_DEVICE_TIMEOUT in a device
+ *     status word that moda_device_status reports; such a kernel skips its
+ *     remaining work and returns instead of hanging.
+ *   - Supported shapes: B, T, Hq, Hkv >= 1, Hq % Hkv == 0, Ld >= 0,
+ *     1 <= d <= 128 for MODA_F32.  MODA_BF16 on the tensor-core path needs
+ *     d == 128 and 128 % G == 0; other bf16 shapes run on the SIMT path
+ *     (d <= 128). Anything else returns MODA_ERR_UNSUPPORTED.
+ *   - Thread safety: entry points may be called concurrently from several
+ *     host threads on different streams.
+ */
+#ifndef MODA_H_
+#define MODA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MODA_ABI_VERSION 1
+
+typedef enum {
+    MODA_OK = 0,
+    MODA_ERR_INVALID_VALUE = 1,   /* NULL pointer, non-positive size, Hq % Hkv != 0 */
+    MODA_ERR_UNSUPPORTED = 2,     /* valid shape this build does not implement      */
+    MODA_ERR_MISALIGNED = 3,      /* a tensor pointer is not 16-byte aligned         */
+    MODA_ERR_WORKSPACE = 4,       /* workspace NULL or smaller than required         */
+    MODA_ERR_LAUNCH = 5,          /* the CUDA launch (or tensor-map encode) failed   */
+    MODA_ERR_DEVICE_TIMEOUT = 6,  /* a kernel's bounded wait expired (device word)   */
+    MODA_ERR_CUDA = 7             /* another CUDA runtime error (device query, sync) */
+} moda_status;
+
+typedef enum { MODA_BF16 = 0, MODA_F32 = 1 } moda_dtype;
+
+/* Kernel family selector for moda_fwd_ex / moda_bwd_ex.  AUTO picks the
+ * tensor-core path when the shape supports it, else SIMT. */
+typedef enum { MODA_IMPL_AUTO = 0, MODA_IMPL_SIMT = 1, MODA_IMPL_TC = 2 } moda_impl;
+
+/* Version of this ABI (MODA_ABI_VERSION of the build). */
+int moda_abi_version(void);
+
+/* Human-readable name of a status code. Never NULL; static storage. */
+const char* moda_status_string(moda_status s);
+
+/*
+ * moda_fwd — fused MoDA forward: causal sequence attention and same-token
+ * depth attention under one online softmax (mhpn.cn §1.2 formula, §2.2 online
+ * softmax and dual mask).
+ *   q    [B,T,Hq,d]        in   queries
+ *   k, v [B,T,Hkv,d]       in   current-layer sequence keys / values
+ *   kd, vd [B,T,Ld,Hkv,d]  in   depth keys / values (NULL iff Ld == 0)
+ *   scale                  in   logit scale, normally 1/sqrt(d); applied to
+ *                               sequence AND depth logits
+ *   out  [B,T,Hq,d]        out  attention output (input dtype)
+ *   lse  [B,Hq,T] fp32     out  natural-log softmax denominator of the scaled
+ *                               logits (needed by moda_bwd); may be NULL
+ * Returns MODA_OK once the kernel is enqueued on `stream`.
+ */
+moda_status moda_fwd(const void* q, const void* k, const void* v,
+                     const void* kd, const void* vd,
+                     int B, int T, int Hq, int Hkv, int d, int Ld,
+                     moda_dtype dtype, float scale,
+                     void* out, float* lse, void* stream);
+
+/* moda_fwd with an explicit kernel family (MODA_IMPL_SIMT forces the scalar
+ * reference kernels; MODA_IMPL_TC requires a tensor-core-supported shape and
+ * returns MODA_ERR_UNSUPPORTED otherwise). Same arguments and semantics. */
+moda_status moda_fwd_ex(const void* q, const void* k, const void* v,
+                        const void* kd, const void* vd,
+                        int B, int T, int Hq, int Hkv, int d, int Ld,
+                        moda_dtype dtype, float scale,
+                        void* out, float* lse, void* stream, moda_impl impl);
+
+/*
+ * moda_bwd_workspace_bytes — bytes of fp32 scratch moda_bwd needs for this
+ * shape (row statistics and, on the tensor-core path, the fp32 dQ
+ * accumulator). Returns 0 for an invalid shape.
+ */
+size_t moda_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int Ld,
+                                moda_dtype dtype);
+
+/*
+ * moda_bwd — gradients of moda_fwd for upstream gradient dout. The pages give
+ * no backward pass; this is the derivative of the forward definition above:
+ *   P = exp(s - lse), D = <dout, out>, dS = P * (dP - D) with
+ *   dP = [dout.v_j || dout.vd_i];  dq = scale*(sum_j dS_j k_j + sum_i dS'_i kd_i),
+ *   dk_j = scale*sum dS_j q, dv_j = sum P_j dout (over rows t >= j of the
+ *   group's G heads), dkd / dvd likewise over the G heads of the same token.
+ *   q,k,v,kd,vd,out   in   as in moda_fwd (out is moda_fwd's output)
+ *   lse               in   moda_fwd's lse
+ *   dout [B,T,Hq,d]   in   upstream gradient
+ *   dq,dk,dv,dkd,dvd  out  gradients, input dtype, same layouts as the inputs
+ *                          (dkd / dvd may be NULL iff Ld == 0)
+ *   workspace         in   device scratch of >= moda_bwd_workspace_bytes(...)
+ *                          bytes, 16-byte aligned; contents on entry ignored
+ */
+moda_status moda_bwd(const void* q, const void* k, const void* v,
+                     const void* kd, const void* vd,
+                     const void* out, const float* lse, const void* dout,
+                     int B, int T, int Hq, int Hkv, int d, int Ld,
+                     moda_dtype dtype, float scale,
+                     void* dq, void* dk, void* dv, void* dkd, void* dvd,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* moda_bwd with an explicit kernel family; same arguments and semantics. */
+moda_status moda_bwd_ex(const void* q, const void* k, const void* v,
+                        const void* kd, const void* vd,
+                        const void* out, const float* lse, const void* dout,
+                        int B, int T, int Hq, int Hkv, int d, int Ld,
+                        moda_dtype dtype, float scale,
+                        void* dq, void* dk, void* dv, void* dkd, void* dvd,
+                        void* workspace, size_t workspace_bytes, void* stream,
+                        moda_impl impl);
+
+/*
+ * moda_pack_depth — optional repack of the depth keys and values into the
+ * flattened per-kv-head layout [2][B][Hkv][T*Ld][d] ("Mixture-of-Depths
+ * Attention", gist.science German summary §2: depth KV flattened along one
+ * T x L axis so that a flash-style kernel reads it blockwise; first half kd,
+ * second half vd). moda_fwd reads the native layout directly, so this is
+ * never needed for correctness; its cost is measured separately.
+ *   kd, vd [B,T,Ld,Hkv,d]  in
+ *   packed                 out  moda_pack_depth_bytes(...) bytes, 16-B aligned
+ */
+size_t moda_pack_depth_bytes(int B, int T, int Hkv, int d, int Ld, moda_dtype dtype);
+moda_status moda_pack_depth(const void* kd, const void* vd,
+                            int B, int T, int Hkv, int d, int Ld, moda_dtype dtype,
+                            void* packed, void* stream);
+
+/* moda_fwd reading depth keys/values from moda_pack_depth's layout. */
+moda_status moda_fwd_packed(const void* q, const void* k, const void* v,
+                            const void* packed_depth,
+                            int B, int T, int Hq, int Hkv, int d, int Ld,
+                            moda_dtype dtype, float scale,
+                            void* out, float* lse, void* stream);
+
+/*
+ * moda_device_status — synchronises `stream`, then reads and clears the
+ * device status word of the current device. Returns MODA_ERR_DEVICE_TIMEOUT if
+ * a kernel's bounded wait expired since the last call, MODA_ERR_CUDA if the
+ * synchronisation itself failed, else MODA_OK.
+ */
+moda_status moda_device_status(void* stream);
+
+/*
+ * moda_debug_set_wait_limit — test hook: caps every bounded on-chip wait of
+ * later launches on the current device at `spins` polls (0 restores the
+ * default, which is far above any legitimate wait). With a tiny cap a wait
+ * that would succeed still expires, which exercises the timeout path without
+ * faulting or hanging the GPU.
+ */
+moda_status moda_debug_set_wait_limit(uint32_t spins);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MODA_H_ */

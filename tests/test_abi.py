@@ -1,0 +1,88 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+that include/moda.h declares, and rejects bad arguments synchronously with
+the documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moda.h")
+
+moda = pytest.importorskip("depth_kv_attention_b200",
+                           reason="libmoda.so not built (python -m depth_kv_attention_b200.build)")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(moda_[a-z0-9_]+)\s*\(",
+                                 src, flags=re.M)))
+
+
+def test_header_declares_the_abi():
+    fns = declared_functions()
+    for name in ["moda_fwd", "moda_bwd", "moda_bwd_workspace_bytes", "moda_pack_depth",
+                 "moda_fwd_packed", "moda_device_status", "moda_status_string"]:
+        assert name in fns
+
+
+def test_every_declared_symbol_is_exported():
+    lib = ctypes.CDLL(moda.LIB_PATH)
+    missing = [f for f in declared_functions() if not hasattr(lib, f)]
+    assert not missing, missing
+
+
+def test_version_and_status_strings():
+    assert moda.moda_abi_version() == 1
+    assert moda.moda_status_string(0) == "MODA_OK"
+    assert moda.moda_status_string(6) == "MODA_ERR_DEVICE_TIMEOUT"
+    assert moda.moda_status_string(99) == "MODA_ERR_UNKNOWN"
+
+
+# Fake, 16-byte aligned "device" addresses: validation rejects the call before
+# any CUDA call or dereference, so they are never used.
+P = 0x10000
+
+
+def fwd(q=P, k=P, v=P, kd=P, vd=P, B=1, T=8, Hq=4, Hkv=2, d=64, Ld=2, dt=0, scale=0.125,
+        out=P, lse=P, impl=0):
+    return moda._c_fwd_ex(q, k, v, kd, vd, B, T, Hq, Hkv, d, Ld, dt, scale, out, lse, None, impl)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(out=None), 1), (dict(kd=None), 1), (dict(vd=None), 1),
+    (dict(B=0), 1), (dict(T=0), 1), (dict(Hq=3, Hkv=2), 1), (dict(Ld=-1), 1), (dict(d=0), 1),
+    (dict(dt=7), 1), (dict(scale=float("nan")), 1), (dict(impl=9), 1),
+    (dict(d=256), 2),
+    (dict(q=P + 2), 3), (dict(kd=P + 8), 3), (dict(lse=P + 4), 3), (dict(out=P + 1), 3),
+])
+def test_fwd_validation(kw, code):
+    assert fwd(**kw) == code
+
+
+def bwd(ws=P, ws_bytes=1 << 30, dq=P, dkd=P, Ld=2, **kw):
+    dims = dict(B=1, T=8, Hq=4, Hkv=2, d=64)
+    dims.update(kw)
+    return moda._c_bwd_ex(P, P, P, P, P, P, P, P, dims["B"], dims["T"], dims["Hq"], dims["Hkv"],
+                          dims["d"], Ld, 0, 0.125, dq, P, P, dkd, P, ws, ws_bytes, None, 0)
+
+
+def test_bwd_validation():
+    assert bwd(ws=None) == 4
+    assert bwd(ws_bytes=16) == 4
+    assert bwd(dq=None) == 1
+    assert bwd(dkd=None) == 1
+    assert bwd(dq=P + 4) == 3
+    assert bwd(ws=P + 8) == 3
+
+
+def test_workspace_and_pack_sizes():
+    # fp32 row statistics [B,Hq,T] (256-byte rounded) + fp32 dQ accumulator for bf16
+    assert moda._c_bwd_ws(1, 8, 4, 2, 64, 2, 0) == 256 + 8 * 4 * 64 * 4
+    assert moda._c_bwd_ws(1, 8, 4, 2, 64, 2, 1) == 256
+    assert moda._c_bwd_ws(1, 8, 3, 2, 64, 2, 0) == 0
+    assert moda._c_pack_bytes(2, 5, 3, 128, 7, 0) == 2 * 2 * 5 * 7 * 3 * 128 * 2
+    assert moda._c_pack(P, P, 1, 4, 1, 128, 2, 0, P + 8, None) == 3
+    assert moda._c_pack(P, P, 1, 4, 1, 6, 2, 0, P, None) == 2
