@@ -1,7 +1,504 @@
-// Tensor-core (tcgen05 / TMEM / TMA) MoDA forward for sm_100a.
+// Tensor-core MoDA forward for sm_100a: TMA -> shared memory -> tcgen05.mma
+// -> TMEM, with the online softmax on the CUDA cores.
+//
+// What it computes: "动态混合深度注意力机制MoDA技术解析" (mhpn.cn) §1.2, one softmax
+// over [Q K_l^T || Q K_depth^T] / sqrt(d) times [V_l || V_depth]; §2.2, the
+// online-softmax state (running max m, running sum "acc" = l, output o)
+// carried across key blocks, with the dual mask (causal over the sequence,
+// same position over depth).
+//
+// How (B200 design, not the pages' kernel):
+//  * Work unit = (b, kv-head, block of 2n tokens), n = 128 / G. It holds two
+//    128-row query tiles; a row is (token, head) in token-major order
+//    (row = token * G + head), so one query tile covers the G heads of a GQA
+//    group for n tokens and every K/V tile is shared by all of them
+//    ("Mixture-of-Depths Attention", gist.science German summary §2,
+//    group-aware indexing).
+//  * Key items: the causal sequence tiles of 128 keys, then the depth chunks.
+//    The depth keys of the unit's tokens are rows t0*Ld .. (t0+2n)*Ld of the
+//    native [B, T*Ld, Hkv, d] view of kd (the flattened T x L axis of the
+//    same summary's flash-compatible layout), loaded 128 rows at a time by
+//    TMA and masked to the row's own token (chunk-aware: only the unit's own
+//    depth range is read). Each depth row is read once per unit.
+//  * Warp roles: warps 0-3 and 4-7 run the softmax of query tiles 0 and 1
+//    (one thread per row, TMEM lane = row); warp 8 issues TMA loads into a
+//    4-stage ring; warp 9 issues tcgen05.mma. TMEM: S0 | S1 | O0 | O1, 128
+//    fp32 columns each; P (bf16) overwrites the first 64 columns of S and is
+//    the TMEM A operand of O += P V. While tile 0's softmax runs, the tensor
+//    core computes tile 1's S, and the other way round.
+//  * Lazy rescaling: the running max used as the exponent reference only
+//    moves when a new row max exceeds it by more than 2^8; O and l use the
+//    same reference, so the final O / l is exact.
+//  * Every mbarrier wait is bounded. On expiry the CTA records
+//    MODA_ERR_DEVICE_TIMEOUT in the device status word, drains its own TMA
+//    loads and MMAs, frees TMEM and exits.
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <cstring>
+
 #include "moda_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace moda {
-bool fwd_tc_supported(const FwdArgs&) { return false; }
-cudaError_t launch_fwd_tc(const FwdArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int kD = 128;                // head dim
+constexpr int kBM = 128;               // rows per query tile
+constexpr int kBN = 128;               // keys per item
+constexpr int kStages = 4;             // K/V ring depth (one tile per stage)
+constexpr int kTileBytes = kBM * kD * 2;       // 32 KB
+constexpr int kHalfBytes = kTileBytes / 2;     // one 64-column swizzled half
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kNoPollLimit = 0;  // drains: time bound only
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct TcFwdParams {
+    CUtensorMap tm_q, tm_k, tm_v, tm_kd, tm_vd;
+    void* out;
+    float* lse;
+    int B, T, Hq, Hkv, G, n, Ld, nblk;
+    float sl2;  // scale * log2(e)
+    int depth_packed;
+    unsigned int* status;
+    unsigned int wait_limit;
+};
+
+struct __align__(8) Bars {
+    uint64_t q_full;
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t s_full[2];
+    uint64_t p_full[2];
+    uint64_t o_final[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+constexpr int kSmemBytes = 2 * kTileBytes + kStages * kTileBytes + 1024 /*bars*/ + 1024 /*align*/;
+
+__device__ __forceinline__ void flag_timeout(TcFwdParams const& p, Bars* bars) {
+    *reinterpret_cast<volatile int*>(&bars->abort_flag) = 1;
+    atomicOr(p.status, 1u);
+}
+
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile_addr, int k16) {
+    // K-major bf16 tile of 128 rows x 128 columns stored as two 128-byte
+    // swizzled halves of 64 columns; step k16 selects columns 16*k16..+15.
+    const uint32_t a = tile_addr + (k16 >> 2) * kHalfBytes + (k16 & 3) * 32;
+    return ptx::umma_desc_sw128(a, 16, 1024);
+}
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile_addr, int k16) {
+    // V tile [128 keys][128 d] as two 64-d swizzled halves: the MMA's N (= d)
+    // is contiguous (MN-major). Step k16 selects keys 16*k16..+15; the two
+    // d-halves are one leading-byte-offset apart, 8-key groups 1024 B apart.
+    const uint32_t a = tile_addr + k16 * 16 * 128;
+    return ptx::umma_desc_sw128(a, kHalfBytes, 1024);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_constant__ TcFwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = smem;                                // 2 tiles
+    uint8_t* sRing = smem + 2 * kTileBytes;            // kStages tiles
+    Bars* bars = reinterpret_cast<Bars*>(sRing + kStages * kTileBytes);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t wait_limit = p.wait_limit;  // 0: time bound only
+    volatile int* abort_flag = &bars->abort_flag;
+
+    // ---- work unit: heaviest (latest) token blocks first
+    const int bh = blockIdx.x % (p.B * p.Hkv);
+    const int tb = p.nblk - 1 - blockIdx.x / (p.B * p.Hkv);
+    const int b = bh / p.Hkv, kvh = bh % p.Hkv;
+    const int n = p.n;
+    const int t0 = tb * 2 * n;
+    int n_kv[2];
+    for (int i = 0; i < 2; ++i) {
+        const int last = min(p.T - 1, t0 + (i + 1) * n - 1);
+        n_kv[i] = last / kBN + 1;
+    }
+    const int n_seq = n_kv[1];
+    const int dep_rows = (min(p.T, t0 + 2 * n) - t0) * p.Ld;
+    const int n_dep = (dep_rows + kBN - 1) / kBN;
+    const int n_items = n_seq + n_dep;
+
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&bars->q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(&bars->full[s], 1);
+            ptx::mbar_init(&bars->empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&bars->s_full[i], 1);
+            ptx::mbar_init(&bars->p_full[i], 128);
+            ptx::mbar_init(&bars->o_final[i], 1);
+        }
+        ptx::mbar_init(&bars->drain, 1);
+        bars->abort_flag = 0;
+        ptx::fence_barrier_init();
+        ptx::fence_proxy_async_smem();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(&bars->tmem_base, 512);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == kProducerWarp) {
+        if (lane == 0) {
+            ptx::prefetch_tmap(&p.tm_q);
+            ptx::prefetch_tmap(&p.tm_k);
+            ptx::prefetch_tmap(&p.tm_v);
+            if (p.Ld > 0) {
+                ptx::prefetch_tmap(&p.tm_kd);
+                ptx::prefetch_tmap(&p.tm_vd);
+            }
+            ptx::mbar_arrive_expect_tx(&bars->q_full, 2 * kTileBytes);
+            for (int i = 0; i < 2; ++i)
+                for (int hf = 0; hf < 2; ++hf)
+                    ptx::tma_load_4d(sQ + i * kTileBytes + hf * kHalfBytes, &p.tm_q, &bars->q_full,
+                                     hf * 64, kvh * p.G, t0 + i * n, b);
+            int seq = 0;
+            bool ok = true;
+            for (int x = 0; x < n_items && ok; ++x) {
+                for (int kv = 0; kv < 2; ++kv, ++seq) {
+                    const int st = seq % kStages;
+                    const uint32_t ph = (seq / kStages) & 1;
+                    if (!ptx::mbar_wait(&bars->empty[st], ph ^ 1, wait_limit, abort_flag)) {
+                        flag_timeout(p, bars);
+                        ok = false;
+                        break;
+                    }
+                    ptx::mbar_arrive_expect_tx(&bars->full[st], kTileBytes);
+                    uint8_t* dst = sRing + st * kTileBytes;
+                    for (int hf = 0; hf < 2; ++hf) {
+                        if (x < n_seq) {
+                            ptx::tma_load_4d(dst + hf * kHalfBytes, kv ? &p.tm_v : &p.tm_k, &bars->full[st],
+                                             hf * 64, kvh, x * kBN, b);
+                        } else {
+                            const int row = t0 * p.Ld + (x - n_seq) * kBN;
+                            const CUtensorMap* m = kv ? &p.tm_vd : &p.tm_kd;
+                            if (p.depth_packed)
+                                ptx::tma_load_4d(dst + hf * kHalfBytes, m, &bars->full[st], hf * 64, row, kvh, b);
+                            else
+                                ptx::tma_load_4d(dst + hf * kHalfBytes, m, &bars->full[st], hf * 64, kvh, row, b);
+                        }
+                    }
+                }
+            }
+            // Drain: every load this CTA issued lands before the CTA can exit.
+            ptx::mbar_wait(&bars->q_full, 0, kNoPollLimit, abort_flag);
+            for (int s = (seq > kStages ? seq - kStages : 0); s < seq; ++s)
+                ptx::mbar_wait(&bars->full[s % kStages], (s / kStages) & 1, kNoPollLimit, abort_flag);
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(kBM, kBN, 0, 0);
+            constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, 0, 1);
+            const uint32_t sQa = ptx::smem_u32(sQ);
+            const uint32_t sRa = ptx::smem_u32(sRing);
+            bool ok = ptx::mbar_wait(&bars->q_full, 0, wait_limit, abort_flag);
+            int cnt_p[2] = {0, 0};
+            auto part = [&](int i, int x) { return x < n_kv[i] || x >= n_seq; };
+            auto wait_full = [&](int seq) {
+                if (!ok) return;
+                if (!ptx::mbar_wait(&bars->full[seq % kStages], (seq / kStages) & 1, wait_limit, abort_flag)) {
+                    flag_timeout(p, bars);
+                    ok = false;
+                }
+                ptx::tc_fence_after();
+            };
+            auto issue_s = [&](int i, int seq) {
+                const uint32_t kt = sRa + (seq % kStages) * kTileBytes;
+                const uint32_t qt = sQa + i * kTileBytes;
+#pragma unroll
+                for (int k = 0; k < kD / 16; ++k)
+                    ptx::mma_ss(tmem + i * 128, desc_kmajor(qt, k), desc_kmajor(kt, k), idesc_qk, k > 0);
+                ptx::mma_commit(&bars->s_full[i]);
+            };
+            if (ok) ptx::tc_fence_after();
+            wait_full(0);
+            if (ok) {
+                for (int i = 0; i < 2; ++i)
+                    if (part(i, 0)) issue_s(i, 0);
+                ptx::mma_commit(&bars->empty[0]);
+            }
+            for (int x = 0; x < n_items && ok; ++x) {
+                const int sv = 2 * x + 1, sk = 2 * x + 2;
+                const bool next = x + 1 < n_items;
+                wait_full(sv);
+                bool k_ready = false;
+                for (int i = 0; i < 2 && ok; ++i) {
+                    if (part(i, x)) {
+                        if (!ptx::mbar_wait(&bars->p_full[i], cnt_p[i] & 1, wait_limit, abort_flag)) {
+                            flag_timeout(p, bars);
+                            ok = false;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        const uint32_t vt = sRa + (sv % kStages) * kTileBytes;
+#pragma unroll
+                        for (int k = 0; k < kBN / 16; ++k)
+                            ptx::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8, desc_mnmajor(vt, k),
+                                        idesc_pv, (cnt_p[i] > 0 || k > 0) ? 1u : 0u);
+                        ++cnt_p[i];
+                    }
+                    if (next && part(i, x + 1)) {
+                        if (!k_ready) {
+                            wait_full(sk);
+                            k_ready = true;
+                            if (!ok) break;
+                        }
+                        issue_s(i, sk);
+                    }
+                }
+                if (!ok) break;
+                ptx::mma_commit(&bars->empty[sv % kStages]);
+                if (next) ptx::mma_commit(&bars->empty[sk % kStages]);
+            }
+            if (ok) {
+                ptx::mma_commit(&bars->o_final[0]);
+                ptx::mma_commit(&bars->o_final[1]);
+            }
+            // Drain: all MMAs issued by this thread complete before TMEM is freed.
+            ptx::mma_commit(&bars->drain);
+            ptx::mbar_wait(&bars->drain, 0, kNoPollLimit, abort_flag);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ softmax warpgroups
+        const int i = warp / 4;            // query tile
+        const int r = (warp % 4) * 32 + lane;  // row = TMEM lane
+        const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
+        const uint32_t tS = tmem + lane_off + i * 128;
+        const uint32_t tO = tmem + lane_off + 256 + i * 128;
+        const int tl = i * n + r / p.G;    // token offset in the unit
+        const int t = t0 + tl;
+        const int h = kvh * p.G + r % p.G;
+        const float sl2 = p.sl2;
+        float m = -INFINITY, l = 0.f;
+        const int n_it = n_kv[i] + n_dep;
+        bool ok = true;
+        for (int it = 0; it < n_it; ++it) {
+            const int x = it < n_kv[i] ? it : it + (n_seq - n_kv[i]);
+            // tcgen05.ld / st below are warp-collective: every decision that
+            // guards them is made warp-uniform.
+            const bool got = ptx::mbar_wait(&bars->s_full[i], it & 1, wait_limit, abort_flag);
+            if (!__all_sync(0xffffffffu, got)) {
+                flag_timeout(p, bars);
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            float s[128];
+            {
+                uint32_t su[128];
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    ptx::tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&su[c * 32]));
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(su[c]);
+            }
+            if (x < n_seq) {
+                const int kbase = x * kBN;
+                if (kbase + kBN - 1 > t) {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (kbase + c > t) s[c] = -INFINITY;
+                }
+            } else {
+                const int lo = tl * p.Ld - (x - n_seq) * kBN;
+                const int hi = lo + p.Ld;
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c < lo || c >= hi) s[c] = -INFINITY;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            const float mxs = mx * sl2;
+            if (__any_sync(0xffffffffu, mxs > m + kRescaleThreshold)) {
+                // Move the exponent reference of every row of the warp to its
+                // running max; rescale l and the O already accumulated (every
+                // earlier P V has completed: S of this item was committed
+                // after it).
+                const float mnew = fmaxf(m, mxs);
+                const float corr = (mnew == -INFINITY) ? 1.f : ptx::ex2(m - mnew);
+                if (it > 0) {
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t o[32];
+                        ptx::tmem_ld32(tO + c * 32, o);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+                        ptx::tmem_st32(tO + c * 32, o);
+                    }
+                }
+                l *= corr;
+                m = mnew;
+            }
+            uint32_t pk[64];
+            float rs = 0.f;
+            const float mref = (m == -INFINITY) ? 0.f : m;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                const float p0 = ptx::ex2(fmaf(s[2 * c], sl2, -mref));
+                const float p1 = ptx::ex2(fmaf(s[2 * c + 1], sl2, -mref));
+                rs += p0 + p1;
+                pk[c] = ptx::pack_bf16x2(p0, p1);
+            }
+            l += rs;
+            ptx::tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
+            ptx::tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&bars->p_full[i]);
+        }
+        if (ok) {
+            const bool got = ptx::mbar_wait(&bars->o_final[i], 0, wait_limit, abort_flag);
+            if (!__all_sync(0xffffffffu, got)) {
+                flag_timeout(p, bars);
+                ok = false;
+            }
+        }
+        ptx::tc_fence_after();
+        if (ok) {
+            const bool valid = t < p.T;
+            const float inv = 1.f / l;
+            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + (((long long)b * p.T + (valid ? t : 0)) * p.Hq + h) * kD;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                ptx::tmem_ld32(tO + c * 32, o);
+                ptx::tmem_wait_ld();
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    w[e] = ptx::pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+                if (valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                }
+            }
+            if (valid && p.lse)
+                p.lse[((long long)b * p.Hq + h) * p.T + t] = (m + __log2f(l)) * 0.6931471805599453f;
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 512);
+    }
+}
+
+// ----------------------------------------------------------------- host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+// 4-D bf16 map, 128-byte swizzle; dims / byte strides innermost first.
+bool make_map(CUtensorMap* m, const void* base, const cuuint64_t dims[4], const cuuint64_t strides_b[3],
+              const cuuint32_t box[4]) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides_b, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool fwd_tc_supported(const FwdArgs& a) {
+    if (a.dtype != MODA_BF16 || a.d != kD) return false;
+    if (a.G < 1 || a.G > 128 || 128 % a.G) return false;
+    // natural q / k / v / out strides (the ABI's layouts)
+    const Strides4 sq = strides_q(a.T, a.Hq, a.d), skv = strides_q(a.T, a.Hkv, a.d);
+    if (a.sq.sb != sq.sb || a.sq.st != sq.st || a.sq.sh != sq.sh) return false;
+    if (a.so.sb != sq.sb || a.so.st != sq.st || a.so.sh != sq.sh) return false;
+    if (a.skv.sb != skv.sb || a.skv.st != skv.st || a.skv.sh != skv.sh) return false;
+    if ((long long)a.T * a.Ld >= (1LL << 31)) return false;  // TMA coordinates are int32
+    return true;
+}
+
+cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s) {
+    TcFwdParams p;
+    memset(&p, 0, sizeof(p));
+    const int G = a.G, n = 128 / G;
+    const cuuint64_t e = 2;  // bytes per bf16
+    {
+        const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)a.Hq, (cuuint64_t)a.T, (cuuint64_t)a.B};
+        const cuuint64_t st[3] = {kD * e, (cuuint64_t)a.Hq * kD * e, (cuuint64_t)a.T * a.Hq * kD * e};
+        const cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)n, 1};
+        if (!make_map(&p.tm_q, a.q, dims, st, box)) return cudaErrorInvalidValue;
+    }
+    {
+        const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)a.Hkv, (cuuint64_t)a.T, (cuuint64_t)a.B};
+        const cuuint64_t st[3] = {kD * e, (cuuint64_t)a.Hkv * kD * e, (cuuint64_t)a.T * a.Hkv * kD * e};
+        const cuuint32_t box[4] = {64, 1, (cuuint32_t)kBN, 1};
+        if (!make_map(&p.tm_k, a.k, dims, st, box)) return cudaErrorInvalidValue;
+        if (!make_map(&p.tm_v, a.v, dims, st, box)) return cudaErrorInvalidValue;
+    }
+    const bool packed = a.Ld > 0 && a.sdep.si == kD;  // [B, Hkv, T*Ld, d]
+    if (a.Ld > 0) {
+        const cuuint64_t rows = (cuuint64_t)a.T * a.Ld;
+        if (packed) {
+            const cuuint64_t dims[4] = {(cuuint64_t)kD, rows, (cuuint64_t)a.Hkv, (cuuint64_t)a.B};
+            const cuuint64_t st[3] = {kD * e, rows * kD * e, (cuuint64_t)a.Hkv * rows * kD * e};
+            const cuuint32_t box[4] = {64, (cuuint32_t)kBN, 1, 1};
+            if (!make_map(&p.tm_kd, a.kd, dims, st, box)) return cudaErrorInvalidValue;
+            if (!make_map(&p.tm_vd, a.vd, dims, st, box)) return cudaErrorInvalidValue;
+        } else {
+            const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)a.Hkv, rows, (cuuint64_t)a.B};
+            const cuuint64_t st[3] = {kD * e, (cuuint64_t)a.Hkv * kD * e, rows * a.Hkv * kD * e};
+            const cuuint32_t box[4] = {64, 1, (cuuint32_t)kBN, 1};
+            if (!make_map(&p.tm_kd, a.kd, dims, st, box)) return cudaErrorInvalidValue;
+            if (!make_map(&p.tm_vd, a.vd, dims, st, box)) return cudaErrorInvalidValue;
+        }
+    } else {
+        p.tm_kd = p.tm_k;
+        p.tm_vd = p.tm_v;
+    }
+    p.out = a.out;
+    p.lse = a.lse;
+    p.B = a.B; p.T = a.T; p.Hq = a.Hq; p.Hkv = a.Hkv; p.G = G; p.n = n; p.Ld = a.Ld;
+    p.nblk = (a.T + 2 * n - 1) / (2 * n);
+    p.sl2 = a.scale * 1.4426950408889634f;
+    p.depth_packed = packed ? 1 : 0;
+    p.status = a.status;
+    p.wait_limit = a.wait_limit;
+    cudaError_t err = cudaFuncSetAttribute(moda_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (err != cudaSuccess) return err;
+    const long long grid = (long long)p.nblk * a.B * a.Hkv;
+    if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+    moda_fwd_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(p);
+    return cudaGetLastError();
+}
+
 }  // namespace moda
