@@ -264,10 +264,15 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-extra", action="store_true", help="skip the Ld=0 and e2e runs")
+    ap.add_argument("--shape", default=None,
+                    help="B,T,Hq,Hkv,d,Ld override of the workload (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
+    if args.shape:
+        B, T, Hq, Hkv, d, Ld = (int(v) for v in args.shape.split(","))
+        w = w.with_(name=f"{w.name}-shape", B=B, T=T, Hq=Hq, Hkv=Hkv, d=d, Ld=Ld)
     if args.impl == "reference":
         return reference_arm(args, w)
 

@@ -4,7 +4,7 @@ Argument marshalling only: every function forwards torch CUDA tensors' device
 pointers and the current CUDA stream to the C entry point of the same name.
 All arithmetic runs in the library's CUDA kernels. There is no CPU fallback:
 importing this package fails if the library has not been built
-(``python -m depth_kv_attention_b200.build``).
+(``python depth_kv_attention_b200/csrc/build.py``).
 
 Layouts (contiguous): q/out/dout [B,T,Hq,d]; k/v [B,T,Hkv,d];
 kd/vd [B,T,Ld,Hkv,d]; lse [B,Hq,T] fp32.
@@ -21,13 +21,13 @@ __all__ = [
     "MODA_OK", "ModaError", "lib", "LIB_PATH", "moda_abi_version", "moda_status_string",
     "moda_fwd", "moda_bwd", "moda_bwd_workspace_bytes", "moda_pack_depth",
     "moda_pack_depth_bytes", "moda_fwd_packed", "moda_device_status",
-    "moda_debug_set_wait_limit", "moda_fwd_from_host",
+    "moda_debug_set_wait_limit", "moda_debug_exp2_poly", "moda_fwd_from_host",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoda.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m depth_kv_attention_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python depth_kv_attention_b200/csrc/build.py` "
         "(the MoDA path has no CPU fallback)")
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -57,6 +57,7 @@ _c_pack = _sig("moda_pack_depth", _i, [_vp, _vp] + [_i] * 5 + [_i, _vp, _vp])
 _c_fwd_packed = _sig("moda_fwd_packed", _i, [_vp] * 4 + _DIMS + [_i, _f, _vp, _vp, _vp])
 _c_dev_status = _sig("moda_device_status", _i, [_vp])
 _c_wait_limit = _sig("moda_debug_set_wait_limit", _i, [ctypes.c_uint32])
+_c_exp2_poly = _sig("moda_debug_exp2_poly", _i, [_vp, _vp, _i, _vp])
 
 
 class ModaError(RuntimeError):
@@ -201,6 +202,16 @@ def moda_device_status(stream=None) -> int:
 
 def moda_debug_set_wait_limit(spins: int) -> None:
     _check(_c_wait_limit(spins), "moda_debug_set_wait_limit")
+
+
+def moda_debug_exp2_poly(x, y=None, stream=None):
+    """Apply the forward kernel's FMA-pipe exp2 to a CUDA fp32 tensor."""
+    _check_tensors(x, y)
+    if y is None:
+        y = torch.empty_like(x)
+    with torch.cuda.device(x.device):
+        _check(_c_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "moda_debug_exp2_poly")
+    return y
 
 
 def moda_fwd_from_host(q, k, v, kd=None, vd=None, scale: float | None = None, device="cuda",

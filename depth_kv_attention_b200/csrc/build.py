@@ -1,6 +1,8 @@
 """Build ``libmoda.so`` (the C-ABI library) in-tree with nvcc for sm_100a.
 
-Usage: ``python -m depth_kv_attention_b200.build [-v] [--force]``.
+Usage: ``python depth_kv_attention_b200/csrc/build.py [-v] [--force] [--ptxas-info]``
+(a plain script, so that it runs without importing the package, whose import
+loads the library).
 
 Each ``csrc/*.cu`` compiles to ``_build/<name>.o`` in parallel (skipped when
 the object is newer than its source and every header); the objects link into
@@ -18,9 +20,9 @@ import shutil
 import subprocess
 import sys
 
-PKG = os.path.dirname(os.path.abspath(__file__))
+CSRC = os.path.dirname(os.path.abspath(__file__))
+PKG = os.path.dirname(CSRC)
 ROOT = os.path.dirname(PKG)
-CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoda.so")
 

@@ -230,6 +230,13 @@ moda_status moda_device_status(void* stream) {
     return MODA_OK;
 }
 
+moda_status moda_debug_exp2_poly(const float* x, float* y, int n, void* stream) {
+    if (n < 0 || (n > 0 && (!x || !y))) return MODA_ERR_INVALID_VALUE;
+    if (n == 0) return MODA_OK;
+    cudaError_t e = launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
+}
+
 moda_status moda_debug_set_wait_limit(uint32_t spins) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MODA_ERR_CUDA;

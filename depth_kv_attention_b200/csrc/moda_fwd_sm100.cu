@@ -22,7 +22,8 @@
 //    depth range is read). Each depth row is read once per unit.
 //  * Warp roles: warps 0-3 and 4-7 run the softmax of query tiles 0 and 1
 //    (one thread per row, TMEM lane = row); warp 8 issues TMA loads into a
-//    4-stage ring; warp 9 issues tcgen05.mma. TMEM: S0 | S1 | O0 | O1, 128
+//    4-stage ring; warp 9 issues tcgen05.mma (warps 10-11 only pad the
+//    third warpgroup for the register reallocation). TMEM: S0 | S1 | O0 | O1, 128
 //    fp32 columns each; P (bf16) overwrites the first 64 columns of S and is
 //    the TMEM A operand of O += P V. While tile 0's softmax runs, the tensor
 //    core computes tile 1's S, and the other way round.
@@ -49,11 +50,20 @@ constexpr int kBN = 128;               // keys per item
 constexpr int kStages = 4;             // K/V ring depth (one tile per stage)
 constexpr int kTileBytes = kBM * kD * 2;       // 32 KB
 constexpr int kHalfBytes = kTileBytes / 2;     // one 64-column swizzled half
-constexpr int kThreads = 320;
+// 3 warpgroups: two softmax warpgroups (one per query tile) and one for the
+// TMA producer warp, the MMA warp and two idle warps. Registers at launch:
+// 384 x 168; after reallocation 2 x 128 x 224 + 128 x 56 = 384 x 168.
+constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kSoftmaxRegs = 224;
+constexpr int kControlRegs = 56;
 constexpr uint32_t kNoPollLimit = 0;  // drains: time bound only
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Of every 8 column pairs of a row, pairs kPolyFrom..7 take exp2 from the
+// FMA-pipe polynomial, the rest from the MUFU unit (which alone would be
+// as busy as the tensor core at d = 128).
+constexpr int kPolyFrom = 5;
 
 struct TcFwdParams {
     CUtensorMap tm_q, tm_k, tm_v, tm_kd, tm_vd;
@@ -151,6 +161,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
     ptx::tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
+    // Register reallocation happens inside each role's branch, so that every
+    // instruction of a role is compiled under that role's register budget.
+    if (warp >= 8) ptx::setmaxnreg_dec<kControlRegs>();
     if (warp == kProducerWarp) {
         if (lane == 0) {
             ptx::prefetch_tmap(&p.tm_q);
@@ -273,8 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
             ptx::mbar_wait(&bars->drain, 0, kNoPollLimit, abort_flag);
         }
         __syncwarp();
-    } else {
+    } else if (warp < 8) {
         // ------------------------------------------------ softmax warpgroups
+        ptx::setmaxnreg_inc<kSoftmaxRegs>();
         const int i = warp / 4;            // query tile
         const int r = (warp % 4) * 32 + lane;  // row = TMEM lane
         const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
@@ -322,9 +336,16 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                 for (int c = 0; c < 128; ++c)
                     if (c < lo || c >= hi) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            float mx;
+            {
+                float mp[8];
 #pragma unroll
-            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+                for (int e = 0; e < 8; ++e) mp[e] = s[e];
+#pragma unroll
+                for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
+                mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                           fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+            }
             const float mxs = mx * sl2;
             if (__any_sync(0xffffffffu, mxs > m + kRescaleThreshold)) {
                 // Move the exponent reference of every row of the warp to its
@@ -348,16 +369,28 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                 m = mnew;
             }
             uint32_t pk[64];
-            float rs = 0.f;
             const float mref = (m == -INFINITY) ? 0.f : m;
+            const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(-mref, -mref);
+            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
-                const float p0 = ptx::ex2(fmaf(s[2 * c], sl2, -mref));
-                const float p1 = ptx::ex2(fmaf(s[2 * c + 1], sl2, -mref));
-                rs += p0 + p1;
-                pk[c] = ptx::pack_bf16x2(p0, p1);
+                const float2 xv = ptx::fma2(make_float2(s[2 * c], s[2 * c + 1]), sl2x2, nm2);
+                float2 pv;
+                if ((c & 7) >= kPolyFrom) {
+                    pv = ptx::exp2_poly2(xv);  // FMA pipe
+                } else {
+                    pv.x = ptx::ex2(xv.x);     // MUFU
+                    pv.y = ptx::ex2(xv.y);
+                }
+                acc[c & 3] = ptx::add2(acc[c & 3], pv);
+                pk[c] = ptx::pack_bf16x2(pv.x, pv.y);
             }
-            l += rs;
+            {
+                const float2 a01 = ptx::add2(acc[0], acc[1]), a23 = ptx::add2(acc[2], acc[3]);
+                const float2 a = ptx::add2(a01, a23);
+                l += a.x + a.y;
+            }
             ptx::tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
             ptx::tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
             ptx::tmem_wait_st();
@@ -404,6 +437,17 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
     }
 }
 
+__global__ void exp2_poly_kernel(const float* x, float* y, int n) {
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i + 1 < n) {
+        const float2 r = ptx::exp2_poly2(make_float2(x[i], x[i + 1]));
+        y[i] = r.x;
+        y[i + 1] = r.y;
+    } else if (i < n) {
+        y[i] = ptx::exp2_poly2(make_float2(x[i], 0.f)).x;
+    }
+}
+
 // ----------------------------------------------------------------- host
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -434,6 +478,12 @@ bool make_map(CUtensorMap* m, const void* base, const cuuint64_t dims[4], const 
 }
 
 }  // namespace
+
+cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t s) {
+    const int pairs = (n + 1) / 2;
+    exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(x, y, n);
+    return cudaGetLastError();
+}
 
 bool fwd_tc_supported(const FwdArgs& a) {
     if (a.dtype != MODA_BF16 || a.d != kD) return false;

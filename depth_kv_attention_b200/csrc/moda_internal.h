@@ -73,5 +73,7 @@ bool fwd_tc_supported(const FwdArgs& a);
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s);
 bool bwd_tc_supported(const BwdArgs& a);
 cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s);
+// The forward's FMA-pipe exp2 applied element-wise (test hook).
+cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t s);
 
 }  // namespace moda

@@ -192,12 +192,66 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
            | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
 
+// Warpgroup register reallocation (all 4 warps of a warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------- math
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// Packed fp32x2 arithmetic (one instruction for two lanes of work).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// 2^x for two lanes on the FMA pipe instead of the MUFU unit, for x <= ~16
+// (inputs below -125 return ~2^-125, i.e. 0 at bf16 / softmax scale).
+// Method: split x = j + f with j = round-to-nearest(x) by the 1.5*2^23
+// magic-number addition (Cody and Waite's argument reduction) so that
+// f is in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients were
+// fitted for this library by weighted least squares (Lawson iteration) on
+// Chebyshev nodes, max relative error 7.5e-5 over [-1/2, 1/2]; then add j to
+// the exponent field.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    const float2 magic = make_float2(12582912.f, 12582912.f);
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 y = add2(x, magic);
+    const float2 r = add2(y, make_float2(-12582912.f, -12582912.f));
+    const float2 f = add2(x, make_float2(-r.x, -r.y));
+    float2 p = fma2(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.2426111400f, 0.2426111400f));
+    p = fma2(p, f, make_float2(0.6932609677f, 0.6932609677f));
+    p = fma2(p, f, make_float2(0.9999280572f, 0.9999280572f));
+    float2 out;
+    out.x = __uint_as_float(__float_as_uint(p.x) + (__float_as_uint(y.x) << 23));
+    out.y = __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(y.y) << 23));
+    return out;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -191,6 +191,14 @@ moda_status moda_device_status(void* stream);
  */
 moda_status moda_debug_set_wait_limit(uint32_t spins);
 
+/*
+ * moda_debug_exp2_poly — test hook: y[i] = 2^x[i] computed by the forward
+ * kernel's FMA-pipe exponential (the share of the softmax exponentials that
+ * does not go to the MUFU unit). x, y: device fp32 arrays of n elements.
+ * Relative error <= 1e-4 for x in [-125, 16]; x < -125 gives ~2^-125.
+ */
+moda_status moda_debug_exp2_poly(const float* x, float* y, int n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

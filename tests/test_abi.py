@@ -11,7 +11,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "moda.h")
 
 moda = pytest.importorskip("depth_kv_attention_b200",
-                           reason="libmoda.so not built (python -m depth_kv_attention_b200.build)")
+                           reason="libmoda.so not built (python depth_kv_attention_b200/csrc/build.py)")
 
 
 def declared_functions():
