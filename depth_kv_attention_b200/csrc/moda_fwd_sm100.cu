@@ -207,9 +207,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                 }
             }
             // Drain: every load this CTA issued lands before the CTA can exit.
-            ptx::mbar_wait(&bars->q_full, 0, kNoPollLimit, abort_flag);
+            ptx::mbar_wait(&bars->q_full, 0, kNoPollLimit, nullptr);
             for (int s = (seq > kStages ? seq - kStages : 0); s < seq; ++s)
-                ptx::mbar_wait(&bars->full[s % kStages], (s / kStages) & 1, kNoPollLimit, abort_flag);
+                ptx::mbar_wait(&bars->full[s % kStages], (s / kStages) & 1, kNoPollLimit, nullptr);
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
             }
             // Drain: all MMAs issued by this thread complete before TMEM is freed.
             ptx::mma_commit(&bars->drain);
-            ptx::mbar_wait(&bars->drain, 0, kNoPollLimit, abort_flag);
+            ptx::mbar_wait(&bars->drain, 0, kNoPollLimit, nullptr);
         }
         __syncwarp();
     } else if (warp < 8) {

@@ -54,7 +54,8 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // Bounded wait on the phase of `bar` with parity `parity`. Gives up (returns
 // false) after `timeout_ns` of wall time, after `max_polls` polls when
 // max_polls != 0 (a test hook), or once another warp of the CTA has raised
-// `abort_flag`.
+// `*abort_flag` (not checked when abort_flag is null: the drains at CTA exit
+// must wait for their own copies and MMAs even after an abort).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t max_polls,
                                           volatile int* abort_flag,
                                           uint64_t timeout_ns = 2000000000ull) {
@@ -62,9 +63,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
+        if (max_polls && i >= max_polls) return false;
         if ((i & 63) == 0) {
-            if (*abort_flag) return false;
-            if (max_polls && i >= max_polls) return false;
+            if (abort_flag && *abort_flag) return false;
             if (globaltimer_ns() - t0 > timeout_ns) return false;
         }
     }

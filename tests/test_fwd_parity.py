@@ -56,10 +56,12 @@ SMALL = [
 ]
 
 
-@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
-def test_small_full(w):
-    for impl in impls_for(w):
-        check_full(w, impl)
+CASES = [(w, impl) for w in SMALL for impl in impls_for(w)]
+
+
+@pytest.mark.parametrize("w,impl", CASES, ids=[f"{w.name}-{i}" for w, i in CASES])
+def test_small_full(w, impl):
+    check_full(w, impl)
 
 
 def test_tiny_f32_workload():
