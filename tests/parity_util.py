@@ -19,8 +19,14 @@ def f64(t) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64) if t.dtype != torch.float64 else t.cpu().numpy()
 
 
-def compare(name, got, want, dtype, what="out"):
-    """Element-wise comparison with the path's tolerance; returns the errors."""
+def compare(name, got, want, dtype, what="out", grad=False):
+    """Element-wise comparison with the path's tolerance; returns the errors.
+
+    ``grad=True`` (gradients stored in bf16): the max-abs bound is the stated
+    one plus one bf16 ulp of the reference, 2^-8 * |want|, because storing a
+    gradient of magnitude |g| in bf16 alone costs up to 2^-9 * |g| — more than
+    2e-2 once |g| > 10, which dK / dV (sums over G*T rows) and dQ under large
+    depth keys reach. The mean-abs bound is unchanged."""
     tol = TOL[dtype]
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
@@ -35,6 +41,11 @@ def compare(name, got, want, dtype, what="out"):
         return float(rel.max())
     err = np.abs(got - want)
     mx, mean = float(err.max()) if err.size else 0.0, float(err.mean()) if err.size else 0.0
-    assert mx <= tol["max_abs"], f"{name}: max-abs {mx:.3e} > {tol['max_abs']}"
+    if grad and dtype == "bf16":
+        allowed = tol["max_abs"] + np.abs(want) * 2.0 ** -8
+        worst = float((err / allowed).max()) if err.size else 0.0
+        assert worst <= 1.0, f"{name}: max-abs {mx:.3e}, {worst:.2f}x the bf16-scaled bound"
+    else:
+        assert mx <= tol["max_abs"], f"{name}: max-abs {mx:.3e} > {tol['max_abs']}"
     assert mean <= tol["mean_abs"], f"{name}: mean-abs {mean:.3e} > {tol['mean_abs']}"
     return mx, mean

@@ -41,7 +41,7 @@ def check_bwd(w, impl, x=None):
     for name, g, r in zip(["dq", "dk", "dv", "dkd", "dvd"], grads, want[:5]):
         if w.Ld == 0 and name in ("dkd", "dvd"):
             continue
-        errs[name] = compare(f"{w.name}/{impl} {name}", f64(g), r, w.dtype)
+        errs[name] = compare(f"{w.name}/{impl} {name}", f64(g), r, w.dtype, grad=True)
         # report error relative to the gradient's rms as well
         rms = float(np.sqrt(np.mean(r ** 2))) or 1.0
         print(f"{w.name}/{impl} {name}: max-abs {errs[name][0]:.2e} rms {rms:.2e}")
@@ -59,10 +59,12 @@ SMALL = [
 ]
 
 
-@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
-def test_bwd_small(w):
-    for impl in impls_for(w):
-        check_bwd(w, impl)
+CASES = [(w, impl) for w in SMALL for impl in impls_for(w)]
+
+
+@pytest.mark.parametrize("w,impl", CASES, ids=[f"{w.name}-{i}" for w, i in CASES])
+def test_bwd_small(w, impl):
+    check_bwd(w, impl)
 
 
 @pytest.mark.parametrize("impl", ["tc", "simt"])
