@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "MODA_OK", "ModaError", "lib", "LIB_PATH", "moda_abi_version", "moda_status_string",
-    "moda_fwd", "moda_bwd", "moda_bwd_workspace_bytes", "moda_pack_depth",
+    "moda_fwd", "moda_bwd", "moda_bwd_workspace_bytes", "moda_bwd_noalloc", "moda_pack_depth",
     "moda_pack_depth_bytes", "moda_fwd_packed", "moda_device_status",
     "moda_debug_set_wait_limit", "moda_debug_exp2_poly", "moda_fwd_from_host",
 ]
@@ -58,6 +58,7 @@ _c_fwd_packed = _sig("moda_fwd_packed", _i, [_vp] * 4 + _DIMS + [_i, _f, _vp, _v
 _c_dev_status = _sig("moda_device_status", _i, [_vp])
 _c_wait_limit = _sig("moda_debug_set_wait_limit", _i, [ctypes.c_uint32])
 _c_exp2_poly = _sig("moda_debug_exp2_poly", _i, [_vp, _vp, _i, _vp])
+_c_bwd_noalloc = _sig("moda_bwd_noalloc", _i, [_vp] * 8 + _DIMS + [_i, _f] + [_vp] * 5 + [_vp])
 
 
 class ModaError(RuntimeError):
@@ -156,6 +157,32 @@ def moda_bwd(q, k, v, kd, vd, out, lse, dout, scale: float | None = None, grads=
                          _ptr(dout), B, T, Hq, Hkv, d, Ld, _DTYPE[q.dtype], scale, _ptr(dq),
                          _ptr(dk), _ptr(dv), _ptr(dkd), _ptr(dvd), _ptr(workspace),
                          workspace.numel(), _stream(stream), _IMPL[impl]), "moda_bwd")
+    return dq, dk, dv, dkd, dvd
+
+
+def moda_bwd_noalloc(q, k, v, kd, vd, out, lse, dout, scale: float | None = None, grads=None,
+                     stream=None):
+    """``moda_bwd_noalloc``: the backward without a workspace argument, for
+    callers that cannot allocate device memory (the library's fixed scratch
+    array holds the row statistics). Output tensors come from ``grads`` or
+    are created here by torch (the C call itself allocates nothing).
+    Returns (dq, dk, dv, dkd, dvd)."""
+    if kd is not None and kd.shape[2] == 0:
+        kd = vd = None
+    _check_tensors(q, k, v, kd, vd, out, lse, dout)
+    B, T, Hq, Hkv, d, Ld = _dims(q, k, kd)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                 None if kd is None else torch.empty_like(kd),
+                 None if vd is None else torch.empty_like(vd))
+    dq, dk, dv, dkd, dvd = grads
+    with torch.cuda.device(q.device):
+        _check(_c_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(kd), _ptr(vd), _ptr(out), _ptr(lse),
+                              _ptr(dout), B, T, Hq, Hkv, d, Ld, _DTYPE[q.dtype], scale, _ptr(dq),
+                              _ptr(dk), _ptr(dv), _ptr(dkd), _ptr(dvd), _stream(stream)),
+               "moda_bwd_noalloc")
     return dq, dk, dv, dkd, dvd
 
 

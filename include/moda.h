@@ -153,6 +153,44 @@ moda_status moda_bwd_ex(const void* q, const void* k, const void* v,
                         moda_impl impl);
 
 /*
+ * moda_bwd_noalloc — moda_bwd for callers that cannot allocate device memory.
+ * The paper has no counterpart to this entry point: it serves how a program
+ * embeds the library, not the MoDA method.
+ *
+ * Who needs it: a caller that owns no device allocator for this library, e.g.
+ * a C / C++ host program that hands over only its input and output buffers,
+ * or a runtime that reserves the whole device for its own memory pool, where
+ * a library's cudaMalloc would fail once the pool has claimed the memory or
+ * would bypass the runtime's accounting. Such a caller cannot supply the
+ * workspace moda_bwd needs.
+ *
+ * What it does: the same gradients as moda_bwd (same arguments minus the
+ * workspace, same layouts, same error codes), computed by the scalar (SIMT)
+ * backward kernels, with the fp32 row statistics D[B, Hq, T] kept in a fixed
+ * array of MODA_NOALLOC_SCRATCH_BYTES bytes compiled into the library. It
+ * calls no cudaMalloc or cudaFree and no allocating routine.
+ *   - Cost: every GPU that loads the library holds that array until exit.
+ *   - Limit: B * Hq * T * 4 bytes must fit in the array; larger problems
+ *     return MODA_ERR_WORKSPACE with nothing launched.
+ *   - Set-up: the first call on each device resolves the array's device
+ *     address (cudaGetSymbolAddress, with that device current). Make that
+ *     first call before any stream capture on the device.
+ *   - Sharing: every call on a device uses the same array, which keeps the
+ *     previous call's contents (nothing needs clearing: the backward writes
+ *     every entry before reading it). Calls whose kernels overlap on the GPU
+ *     (different streams without ordering between them) race on the array;
+ *     order them on one stream or with events.
+ */
+#define MODA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+moda_status moda_bwd_noalloc(const void* q, const void* k, const void* v,
+                             const void* kd, const void* vd,
+                             const void* out, const float* lse, const void* dout,
+                             int B, int T, int Hq, int Hkv, int d, int Ld,
+                             moda_dtype dtype, float scale,
+                             void* dq, void* dk, void* dv, void* dkd, void* dvd,
+                             void* stream);
+
+/*
  * moda_pack_depth — optional repack of the depth keys and values into the
  * flattened per-kv-head layout [2][B][Hkv][T*Ld][d] ("Mixture-of-Depths
  * Attention", gist.science German summary §2: depth KV flattened along one
