@@ -137,8 +137,14 @@ def forward_rows(q, k, v, kd, vd, scale: float, b: int, h: int, ts):
     return vals, l
 
 
-def backward(q, k, v, kd, vd, dout, scale: float, row_block: int = 256):
+def backward(q, k, v, kd, vd, dout, scale: float, row_block: int = 256, out_for_D=None):
     """Gradients of the MoDA forward for upstream gradient ``dout``.
+
+    ``out_for_D`` (optional, [B,T,Hq,d]): the forward output to form
+    D = <dout, out> from. By default D uses the exact float64 forward output,
+    which makes the result the exact derivative. A backward that receives the
+    forward output as stored (e.g. rounded to bf16) forms D from that stored
+    output instead; passing it here gives the oracle of that definition.
 
     The pages describe no backward pass; this is the derivative of the
     forward definition above (softmax Jacobian), written per row block:
@@ -156,6 +162,7 @@ def backward(q, k, v, kd, vd, dout, scale: float, row_block: int = 256):
     q, k, v, kd, vd, dout = (to_f64(x) for x in (q, k, v, kd, vd, dout))
     B, T, Hq, Hkv, G, d, Ld = _dims(q, k, kd)
     out, lse = forward(q, k, v, kd, vd, scale, row_block)
+    outD = out if out_for_D is None else to_f64(out_for_D)
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
@@ -171,7 +178,7 @@ def backward(q, k, v, kd, vd, dout, scale: float, row_block: int = 256):
                 dor = dout[b, t0:t1, h]
                 s = _concat_logits(qr, k[b, :t1, g], kd[b, t0:t1, :, g], scale, ts)
                 P = np.exp(s - lse[b, h, t0:t1][:, None])
-                D = np.sum(dor * out[b, t0:t1, h], axis=1)
+                D = np.sum(dor * outD[b, t0:t1, h], axis=1)
                 dP_seq = dor @ v[b, :t1, g].T
                 dP_dep = np.einsum("rc,ric->ri", dor, vd[b, t0:t1, :, g])
                 dP = np.concatenate([dP_seq, dP_dep], axis=1)

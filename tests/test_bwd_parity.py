@@ -21,6 +21,7 @@ def impls_for(w):
 
 
 _ORACLE = {}  # the last workload's oracle gradients, shared by its impl variants
+_LAST_GRADS = [None]
 
 
 def check_bwd(w, impl, x=None):
@@ -33,9 +34,16 @@ def check_bwd(w, impl, x=None):
                           w.scale, impl=impl)
     torch.cuda.synchronize()
     assert moda.moda_device_status() == 0
+    _LAST_GRADS[0] = grads
     if w.name not in _ORACLE:
         _ORACLE.clear()
-        _ORACLE[w.name] = oracle.backward(x["q"], x["k"], x["v"], x["kd"], x["vd"], x["dout"], w.scale)
+        # moda_bwd forms D = <dout, out> from the output it is given, which the
+        # forward stored in the input dtype: the oracle forms D the same way,
+        # from its own forward output rounded to that dtype.
+        ro, _ = oracle.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], w.scale)
+        stored = torch.from_numpy(ro).to(x["q"].dtype)
+        _ORACLE[w.name] = oracle.backward(x["q"], x["k"], x["v"], x["kd"], x["vd"], x["dout"],
+                                          w.scale, out_for_D=stored)
     want = _ORACLE[w.name]
     errs = {}
     for name, g, r in zip(["dq", "dk", "dv", "dkd", "dvd"], grads, want[:5]):
@@ -69,8 +77,15 @@ def test_bwd_small(w, impl):
 
 @pytest.mark.parametrize("impl", ["tc", "simt"])
 def test_bwd_g32_workload_full(impl):
-    """The wide-GQA forward+backward workload (T=8192, G=32, Ld=28), full."""
+    """The wide-GQA forward+backward workload (T=8192, G=32, Ld=28), full,
+    against the oracle of the stored-output definition and, end to end,
+    against the exact derivative (D from the exact forward output)."""
     w = WORKLOADS["g32_fwdbwd"]
     if impl not in impls_for(w):
         pytest.skip("shape not on this path")
-    check_bwd(w, impl)
+    x = make_inputs(w, with_dout=True)
+    check_bwd(w, impl, x)
+    grads = _LAST_GRADS[0]
+    exact = oracle.backward(x["q"], x["k"], x["v"], x["kd"], x["vd"], x["dout"], w.scale)
+    for name, g, r in zip(["dq", "dk", "dv", "dkd", "dvd"], grads, exact[:5]):
+        compare(f"{w.name}/{impl} {name} vs exact derivative", f64(g), r, w.dtype, grad=True)

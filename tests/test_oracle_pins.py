@@ -304,3 +304,29 @@ def test_planted_mistakes_are_caught(monkeypatch):
     assert not _pins_pass()
     monkeypatch.setattr(om, "_softmax_rows", orig_sm)
     assert _pins_pass()
+
+
+def test_backward_with_stored_output_shifts_by_the_D_error():
+    """With D formed from a perturbed forward output out + delta, every row's
+    dS changes by -P * <dout, delta>, so dq changes by
+    -scale * <dout, delta> * (sum_j P_j k_j + sum_i P'_i kd_i) (P from the
+    exact forward), dv and dvd do not change at all."""
+    x, scale = rand_case(1, 6, 2, 1, 4, 3, seed=21, depth_std=2.0)
+    base = om.backward(x["q"], x["k"], x["v"], x["kd"], x["vd"], x["dout"], scale)
+    delta = np.random.default_rng(3).standard_normal(x["q"].shape) * 1e-2
+    pert = om.backward(x["q"], x["k"], x["v"], x["kd"], x["vd"], x["dout"], scale,
+                       out_for_D=base[5] + delta)
+    np.testing.assert_allclose(pert[2], base[2], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(pert[4], base[4], rtol=0, atol=1e-14)
+    lse = base[6]
+    for h in range(2):
+        for t in range(6):
+            qv = x["q"][0, t, h]
+            dD = float(np.dot(x["dout"][0, t, h], delta[0, t, h]))
+            acc = np.zeros(4)
+            for j in range(t + 1):
+                acc += math.exp(scale * float(qv @ x["k"][0, j, 0]) - lse[0, h, t]) * x["k"][0, j, 0]
+            for i in range(3):
+                acc += math.exp(scale * float(qv @ x["kd"][0, t, i, 0]) - lse[0, h, t]) * x["kd"][0, t, i, 0]
+            np.testing.assert_allclose(pert[0][0, t, h] - base[0][0, t, h], -scale * dD * acc,
+                                       rtol=0, atol=1e-12)
