@@ -82,11 +82,14 @@ moda_status run_fwd(FwdArgs& a, void* stream, moda_impl impl) {
     return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
 }
 
-size_t bwd_ws_bytes(int B, int T, int Hq, int d, bool with_dq_acc) {
-    size_t rowD = (size_t)B * Hq * T * sizeof(float);
-    rowD = (rowD + 255) & ~size_t(255);
-    size_t acc = with_dq_acc ? (size_t)B * T * Hq * d * sizeof(float) : 0;
-    return rowD + acc;
+// Workspace: [fp32 D, B*Hq*T, rounded to 256 B] then, for bf16 (tensor-core
+// path), the fp32 accumulators of dq [B,T,Hq,d], dk and dv [B,T,Hkv,d].
+size_t bwd_ws_rowD_bytes(int B, int T, int Hq) {
+    return ((size_t)B * Hq * T * sizeof(float) + 255) & ~size_t(255);
+}
+size_t bwd_ws_bytes(int B, int T, int Hq, int Hkv, int d, bool with_acc) {
+    size_t acc = with_acc ? (size_t)B * T * (Hq + 2 * Hkv) * d * sizeof(float) : 0;
+    return bwd_ws_rowD_bytes(B, T, Hq) + acc;
 }
 
 }  // namespace
@@ -133,9 +136,9 @@ moda_status moda_fwd(const void* q, const void* k, const void* v, const void* kd
 size_t moda_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dtype) {
     if (check_dims(B, T, Hq, Hkv, d, Ld) != MODA_OK) return 0;
     if (dtype != MODA_BF16 && dtype != MODA_F32) return 0;
-    // The fp32 dQ accumulator is reserved for every bf16 shape so that the
+    // The fp32 accumulators are reserved for every bf16 shape so that the
     // size does not depend on which kernel family a call selects.
-    return bwd_ws_bytes(B, T, Hq, d, dtype == MODA_BF16);
+    return bwd_ws_bytes(B, T, Hq, Hkv, d, dtype == MODA_BF16);
 }
 
 moda_status moda_bwd_ex(const void* q, const void* k, const void* v, const void* kd, const void* vd,
@@ -160,8 +163,12 @@ moda_status moda_bwd_ex(const void* q, const void* k, const void* v, const void*
     if (!aligned16(workspace)) return MODA_ERR_MISALIGNED;
     a.dout = dout; a.dq = dq; a.dk = dk; a.dv = dv; a.dkd = dkd; a.dvd = dvd;
     a.rowD = static_cast<float*>(workspace);
-    const size_t rowD = bwd_ws_bytes(B, T, Hq, d, false);
-    a.dq_acc = dtype == MODA_BF16 ? reinterpret_cast<float*>(static_cast<char*>(workspace) + rowD) : nullptr;
+    if (dtype == MODA_BF16) {
+        char* base = static_cast<char*>(workspace) + bwd_ws_rowD_bytes(B, T, Hq);
+        a.dq_acc = reinterpret_cast<float*>(base);
+        a.dk_acc = a.dq_acc + (size_t)B * T * Hq * d;
+        a.dv_acc = a.dk_acc + (size_t)B * T * Hkv * d;
+    }
     cudaError_t e = status_ptr(&a.f.status, &a.f.wait_limit);
     if (e != cudaSuccess) return MODA_ERR_CUDA;
     const bool tc_ok = bwd_tc_supported(a);

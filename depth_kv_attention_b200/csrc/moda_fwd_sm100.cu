@@ -40,6 +40,7 @@
 
 #include "moda_internal.h"
 #include "sm100_ptx.cuh"
+#include "tmap_host.h"
 
 namespace moda {
 namespace {
@@ -448,35 +449,6 @@ __global__ void exp2_poly_kernel(const float* x, float* y, int n) {
     }
 }
 
-// ----------------------------------------------------------------- host
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    }
-    return fn;
-}
-
-// 4-D bf16 map, 128-byte swizzle; dims / byte strides innermost first.
-bool make_map(CUtensorMap* m, const void* base, const cuuint64_t dims[4], const cuuint64_t strides_b[3],
-              const cuuint32_t box[4]) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    const cuuint32_t es[4] = {1, 1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides_b, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t s) {
@@ -506,14 +478,14 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s) {
         const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)a.Hq, (cuuint64_t)a.T, (cuuint64_t)a.B};
         const cuuint64_t st[3] = {kD * e, (cuuint64_t)a.Hq * kD * e, (cuuint64_t)a.T * a.Hq * kD * e};
         const cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)n, 1};
-        if (!make_map(&p.tm_q, a.q, dims, st, box)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16_4d(&p.tm_q, a.q, dims, st, box)) return cudaErrorInvalidValue;
     }
     {
         const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)a.Hkv, (cuuint64_t)a.T, (cuuint64_t)a.B};
         const cuuint64_t st[3] = {kD * e, (cuuint64_t)a.Hkv * kD * e, (cuuint64_t)a.T * a.Hkv * kD * e};
         const cuuint32_t box[4] = {64, 1, (cuuint32_t)kBN, 1};
-        if (!make_map(&p.tm_k, a.k, dims, st, box)) return cudaErrorInvalidValue;
-        if (!make_map(&p.tm_v, a.v, dims, st, box)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16_4d(&p.tm_k, a.k, dims, st, box)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16_4d(&p.tm_v, a.v, dims, st, box)) return cudaErrorInvalidValue;
     }
     const bool packed = a.Ld > 0 && a.sdep.si == kD;  // [B, Hkv, T*Ld, d]
     if (a.Ld > 0) {
@@ -522,14 +494,14 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s) {
             const cuuint64_t dims[4] = {(cuuint64_t)kD, rows, (cuuint64_t)a.Hkv, (cuuint64_t)a.B};
             const cuuint64_t st[3] = {kD * e, rows * kD * e, (cuuint64_t)a.Hkv * rows * kD * e};
             const cuuint32_t box[4] = {64, (cuuint32_t)kBN, 1, 1};
-            if (!make_map(&p.tm_kd, a.kd, dims, st, box)) return cudaErrorInvalidValue;
-            if (!make_map(&p.tm_vd, a.vd, dims, st, box)) return cudaErrorInvalidValue;
+            if (!make_tmap_bf16_4d(&p.tm_kd, a.kd, dims, st, box)) return cudaErrorInvalidValue;
+            if (!make_tmap_bf16_4d(&p.tm_vd, a.vd, dims, st, box)) return cudaErrorInvalidValue;
         } else {
             const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)a.Hkv, rows, (cuuint64_t)a.B};
             const cuuint64_t st[3] = {kD * e, (cuuint64_t)a.Hkv * kD * e, rows * a.Hkv * kD * e};
             const cuuint32_t box[4] = {64, 1, (cuuint32_t)kBN, 1};
-            if (!make_map(&p.tm_kd, a.kd, dims, st, box)) return cudaErrorInvalidValue;
-            if (!make_map(&p.tm_vd, a.vd, dims, st, box)) return cudaErrorInvalidValue;
+            if (!make_tmap_bf16_4d(&p.tm_kd, a.kd, dims, st, box)) return cudaErrorInvalidValue;
+            if (!make_tmap_bf16_4d(&p.tm_vd, a.vd, dims, st, box)) return cudaErrorInvalidValue;
         }
     } else {
         p.tm_kd = p.tm_k;
