@@ -238,6 +238,56 @@ def workload_config(w):
             "parallelism": "replicas"}
 
 
+def make_step(moda, w, x, mode, kernel):
+    """The timed step on device-resident inputs: one forward, or forward and
+    backward. Returns (step, launches of this library's kernels per step,
+    out, lse)."""
+    out = torch.empty_like(x["q"])
+    lse = torch.empty((w.B, w.Hq, w.T), device="cuda", dtype=torch.float32)
+    if mode == "fwd":
+        def step():
+            moda.moda_fwd(x["q"], x["k"], x["v"], x["kd"], x["vd"], w.scale, out=out, lse=lse,
+                          impl=kernel)
+        return step, 1, out, lse
+    grads = (torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"]),
+             torch.empty_like(x["kd"]) if w.Ld else None, torch.empty_like(x["vd"]) if w.Ld else None)
+    ws = torch.empty(max(16, moda.moda_bwd_workspace_bytes(w.B, w.T, w.Hq, w.Hkv, w.d, w.Ld,
+                                                            x["q"].dtype)),
+                     device="cuda", dtype=torch.uint8)
+
+    def step():
+        moda.moda_fwd(x["q"], x["k"], x["v"], x["kd"], x["vd"], w.scale, out=out, lse=lse,
+                      impl=kernel)
+        moda.moda_bwd(x["q"], x["k"], x["v"], x["kd"], x["vd"], out, lse, x["dout"], w.scale,
+                      grads=grads, workspace=ws, impl=kernel)
+    # forward 1; backward: D, depth dq, depth dk/dv (Ld > 0), sequence, 3 conversions
+    return step, 1 + 6 + (1 if w.Ld else 0), out, lse
+
+
+def measure_secondary(moda, w, world, kernel, steps=5, warmup=3):
+    """Forward TFLOP/s and overhead vs Ld = 0 of another workload; for the
+    forward+backward workload also the backward time and fwd+bwd TFLOP/s."""
+    x = {k: v.cuda() for k, v in make_inputs(w, with_dout=w.backward).items()}
+    step, _, out, lse = make_step(moda, w, x, "fwd", kernel)
+    ms, _ = timed(step, steps, warmup, world)
+    x0 = dict(x, kd=None, vd=None)
+    w0 = w.with_(Ld=0)
+    step0, _, _, _ = make_step(moda, w0, x0, "fwd", kernel)
+    ms0, _ = timed(step0, steps, warmup, world)
+    res = {"config": f"B={w.B} T={w.T} Hq={w.Hq} Hkv={w.Hkv} d={w.d} Ld={w.Ld}",
+           "fwd_ms": ms, "fwd_tflops": credited_flops(w) / (ms * 1e-3) / 1e12,
+           "ld0_fwd_ms": ms0, "overhead_vs_ld0": ms / ms0 - 1.0}
+    if w.backward:
+        stepb, _, _, _ = make_step(moda, w, x, "fwdbwd", kernel)
+        msb, _ = timed(stepb, steps, warmup, world)
+        res.update({"fwd_bwd_ms": msb, "bwd_ms": msb - ms,
+                    "bwd_tflops": 2.5 * credited_flops(w) / ((msb - ms) * 1e-3) / 1e12,
+                    "fwd_bwd_tflops": 3.5 * credited_flops(w) / (msb * 1e-3) / 1e12})
+    del x
+    torch.cuda.empty_cache()
+    return res
+
+
 def traffic_for(kernel_src: str):
     """DRAM bytes per launch from the committed ncu summary, or None when the
     kernel source changed since the counters were taken."""
@@ -264,6 +314,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-extra", action="store_true", help="skip the Ld=0 and e2e runs")
+    ap.add_argument("--mode", default="fwd", choices=["fwd", "fwdbwd"],
+                    help="step = forward, or forward + backward (credited 3.5x the forward FLOPs)")
     ap.add_argument("--shape", default=None,
                     help="B,T,Hq,Hkv,d,Ld override of the workload (profiling runs)")
     args = ap.parse_args()
@@ -280,29 +332,23 @@ def main():
 
     world, rank, local = dist_setup(args.gpus)
     peaks, peaks_kind = load_peaks()
-    x_host = make_inputs(w)
+    x_host = make_inputs(w, with_dout=args.mode == "fwdbwd")
     x = {k: v.cuda() for k, v in x_host.items()}
-    out = torch.empty_like(x["q"])
-    lse = torch.empty((w.B, w.Hq, w.T), device="cuda", dtype=torch.float32)
-
-    def step():
-        moda.moda_fwd(x["q"], x["k"], x["v"], x["kd"], x["vd"], w.scale, out=out, lse=lse,
-                      impl=args.kernel)
+    step, launches_per_step, out, lse = make_step(moda, w, x, args.mode, args.kernel)
 
     step()
     torch.cuda.synchronize()
     if moda.moda_device_status() != 0:
-        raise RuntimeError("device status word set after the first forward")
+        raise RuntimeError("device status word set after the first step")
     clocks = ClockSampler(local)
     clocks.start()
     ms, launch_ms = timed(step, args.steps, args.warmup, world)
     clk = clocks.stop()
-    flops = credited_flops(w)
+    flops = credited_flops(w) * (3.5 if args.mode == "fwdbwd" else 1.0)
     value = flops * world / (ms * 1e-3) / 1e12
-    launches_per_step = 1
 
     extra = {}
-    if not args.no_extra:
+    if not args.no_extra and args.mode == "fwd" and not args.shape:
         # the same library's own causal attention with Ld = 0
         out0 = torch.empty_like(out)
 
@@ -315,7 +361,7 @@ def main():
         del out0
 
     e2e = None
-    if not args.no_extra:
+    if not args.no_extra and args.mode == "fwd":
         pinned = {k: v.pin_memory() for k, v in x_host.items()}
         out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
@@ -341,8 +387,12 @@ def main():
                 "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                 "frac_of_nominal_2250": achieved / 2250.0}
 
+    if not args.no_extra and not args.shape:
+        extra["other_workloads"] = {name: measure_secondary(moda, WORKLOADS[name], world, args.kernel)
+                                    for name in ("t4k", "t16k_b2", "g32_fwdbwd") if name != w.name}
+
     cpu = None
-    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+    if rank == 0 and world == 1 and args.cpu_seconds > 0 and args.mode == "fwd":
         tf, nrows, secs = oracle_sample(w, args.cpu_seconds, x_host)
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"{nrows} seed-sampled query rows (64 per (b, head), heads in turn) "
@@ -357,6 +407,7 @@ def main():
             "pct_of_bf16_peak": 100.0 * value / world / peak,
             "clocks": clk, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
             "roofline": roofline, "cpu_baseline": cpu, "kernel_family": args.kernel,
+            "mode": args.mode,
         }
         line.update(extra)
         print(json.dumps(line), flush=True)

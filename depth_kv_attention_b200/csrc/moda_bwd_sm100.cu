@@ -86,14 +86,6 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t tile, int k16) {
     return ptx::umma_desc_sw128(tile + k16 * 16 * 128, kHalf, 1024);
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
@@ -137,17 +129,22 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_seq_tc_kernel(const __gr
     const uint32_t wait_limit = p.wait_limit;
     volatile int* abort_flag = &bars->abort_flag;
 
-    // Work item: (b, kv-head) = blockIdx.z, key tile = blockIdx.y, and a chunk
-    // of at most qchunk query tiles = blockIdx.x. Key tiles near the start see
-    // more query tiles; their chunks past the end exit at once.
+    // Work item: key tile = blockIdx.x (fastest), chunk of query tokens =
+    // blockIdx.y, (b, kv-head) = blockIdx.z. A chunk is qchunk query tiles of
+    // absolute token range [c*qchunk*n, (c+1)*qchunk*n); the CTAs in flight
+    // at one time are the key tiles of one or two chunks, so their fp32 dq
+    // reductions land on the same few MB of dq rows (L2-resident). Key tiles
+    // that no row of the chunk can see exit at once.
     const int b = blockIdx.z / p.Hkv, kvh = blockIdx.z % p.Hkv;
-    const int kt = blockIdx.y;
+    const int kt = blockIdx.x;
     const int j0 = kt * kBK;
     const int n = p.n;
-    const int nq_all = (p.T - j0 + n - 1) / n;
-    const int q_first = blockIdx.x * p.qchunk;
-    if (q_first >= nq_all) return;
-    const int nq = min(p.qchunk, nq_all - q_first);
+    const int c_lo = blockIdx.y * p.qchunk * n;                      // first token of the chunk
+    const int c_hi = min(p.T, (blockIdx.y + 1) * p.qchunk * n);      // one past its last token
+    const int t_first = max(j0, c_lo);                               // multiple of n
+    if (t_first >= c_hi) return;
+    const int nq = (c_hi - t_first + n - 1) / n;
+    const int q_first = (t_first - j0) / n;                          // query tiles counted from j0
 
     if (threadIdx.x == 0) {
         ptx::mbar_init(&bars->kv_full, 1);
@@ -322,8 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_seq_tc_kernel(const __gr
                     pp[e2] = ptx::pack_bf16x2(pv[0], pv[1]);
                     dd[e2] = ptx::pack_bf16x2(dv[0], dv[1]);
                 }
-                tmem_st16(tmem + lane_off + 0 + 16 * c, pp);
-                tmem_st16(tmem + lane_off + 128 + 16 * c, dd);
+                ptx::tmem_st16(tmem + lane_off + 0 + 16 * c, pp);
+                ptx::tmem_st16(tmem + lane_off + 128 + 16 * c, dd);
                 // dS into shared memory, [key][row] with rows contiguous (the
                 // MN-major A operand of dQ = dS K), 128-byte swizzle.
                 uint8_t* half = sDS + (c >> 1) * kHalf + r * 128;
@@ -561,8 +558,8 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s) {
     const size_t kv_bytes = (size_t)f.B * f.T * f.Hkv * kD * sizeof(float);
     if ((e = cudaMemsetAsync(a.dk_acc, 0, kv_bytes, s)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(a.dv_acc, 0, kv_bytes, s)) != cudaSuccess) return e;
-    const int max_chunks = ((f.T + n - 1) / n + p.qchunk - 1) / p.qchunk;
-    dim3 grid(max_chunks, p.nkt, f.B * f.Hkv);
+    const int n_chunks = ((f.T + n - 1) / n + p.qchunk - 1) / p.qchunk;
+    dim3 grid(p.nkt, n_chunks, f.B * f.Hkv);
     moda_bwd_seq_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 

@@ -48,23 +48,32 @@ namespace {
 constexpr int kD = 128;                // head dim
 constexpr int kBM = 128;               // rows per query tile
 constexpr int kBN = 128;               // keys per item
-constexpr int kStages = 4;             // K/V ring depth (one tile per stage)
+constexpr int kStages = 5;             // K/V ring depth (one tile per stage)
 constexpr int kTileBytes = kBM * kD * 2;       // 32 KB
 constexpr int kHalfBytes = kTileBytes / 2;     // one 64-column swizzled half
 // 3 warpgroups: two softmax warpgroups (one per query tile) and one for the
 // TMA producer warp, the MMA warp and two idle warps. Registers at launch:
-// 384 x 168; after reallocation 2 x 128 x 224 + 128 x 56 = 384 x 168.
+// 384 x 168; after reallocation 2 x 128 x 216 + 128 x 72 = 384 x 168.
 constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kSoftmaxRegs = 224;
-constexpr int kControlRegs = 56;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kControlRegs = 72;
 constexpr uint32_t kNoPollLimit = 0;  // drains: time bound only
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Of every 8 column pairs of a row, pairs kPolyFrom..7 take exp2 from the
 // FMA-pipe polynomial, the rest from the MUFU unit (which alone would be
 // as busy as the tensor core at d = 128).
-constexpr int kPolyFrom = 5;
+#ifndef MODA_POLY_FROM
+#define MODA_POLY_FROM 8
+#endif
+constexpr int kPolyFrom = MODA_POLY_FROM;
+// P is handed to the PV MMA in this many chunks (128 / kPChunks keys each).
+#ifndef MODA_PCHUNKS
+#define MODA_PCHUNKS 1
+#endif
+constexpr int kPChunks = MODA_PCHUNKS;
+static_assert(kPChunks == 1 || kPChunks == 2 || kPChunks == 4, "P chunks");
 
 struct TcFwdParams {
     CUtensorMap tm_q, tm_k, tm_v, tm_kd, tm_vd;
@@ -82,7 +91,7 @@ struct __align__(8) Bars {
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t s_full[2];
-    uint64_t p_full[2];
+    uint64_t p_full[2][4];  // [tile][P chunk]
     uint64_t o_final[2];
     uint64_t drain;
     uint32_t tmem_base;
@@ -90,24 +99,12 @@ struct __align__(8) Bars {
 };
 
 constexpr int kSmemBytes = 2 * kTileBytes + kStages * kTileBytes + 1024 /*bars*/ + 1024 /*align*/;
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+static_assert(sizeof(Bars) <= 1024, "barrier block");
 
 __device__ __forceinline__ void flag_timeout(TcFwdParams const& p, Bars* bars) {
     *reinterpret_cast<volatile int*>(&bars->abort_flag) = 1;
     atomicOr(p.status, 1u);
-}
-
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile_addr, int k16) {
-    // K-major bf16 tile of 128 rows x 128 columns stored as two 128-byte
-    // swizzled halves of 64 columns; step k16 selects columns 16*k16..+15.
-    const uint32_t a = tile_addr + (k16 >> 2) * kHalfBytes + (k16 & 3) * 32;
-    return ptx::umma_desc_sw128(a, 16, 1024);
-}
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile_addr, int k16) {
-    // V tile [128 keys][128 d] as two 64-d swizzled halves: the MMA's N (= d)
-    // is contiguous (MN-major). Step k16 selects keys 16*k16..+15; the two
-    // d-halves are one leading-byte-offset apart, 8-key groups 1024 B apart.
-    const uint32_t a = tile_addr + k16 * 16 * 128;
-    return ptx::umma_desc_sw128(a, kHalfBytes, 1024);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_constant__ TcFwdParams p) {
@@ -127,15 +124,25 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
     const int b = bh / p.Hkv, kvh = bh % p.Hkv;
     const int n = p.n;
     const int t0 = tb * 2 * n;
-    int n_kv[2];
+    // Items: the causal sequence tiles of 128 keys, then the depth chunks:
+    // 128-row slices of the unit's depth rows t0*Ld .. (t0+2n)*Ld of the
+    // [B, T*Ld, Hkv, d] view. Every item occupies two ring slots (K, V).
+    int n_kv[2], nv[2];
     for (int i = 0; i < 2; ++i) {
         const int last = min(p.T - 1, t0 + (i + 1) * n - 1);
         n_kv[i] = last / kBN + 1;
+        nv[i] = max(0, min(n, p.T - t0 - i * n));  // tokens of tile i inside the sequence
     }
     const int n_seq = n_kv[1];
-    const int dep_rows = (min(p.T, t0 + 2 * n) - t0) * p.Ld;
-    const int n_dep = (dep_rows + kBN - 1) / kBN;
+    const int n_dep = ((nv[0] + nv[1]) * p.Ld + kBN - 1) / kBN;
     const int n_items = n_seq + n_dep;
+    // Tile i takes part in sequence items up to its last token's tile, and in
+    // the depth chunks that overlap its own tokens' depth rows.
+    auto part = [&](int i, int x) {
+        if (x < n_seq) return x < n_kv[i];
+        const int lo = (x - n_seq) * kBN, row0 = i * n * p.Ld;
+        return nv[i] > 0 && lo < row0 + nv[i] * p.Ld && lo + kBN > row0;
+    };
 
     if (threadIdx.x == 0) {
         ptx::mbar_init(&bars->q_full, 1);
@@ -145,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&bars->s_full[i], 1);
-            ptx::mbar_init(&bars->p_full[i], 128);
+            for (int c = 0; c < kPChunks; ++c) ptx::mbar_init(&bars->p_full[i][c], 128);
             ptx::mbar_init(&bars->o_final[i], 1);
         }
         ptx::mbar_init(&bars->drain, 1);
@@ -166,7 +173,10 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
     // instruction of a role is compiled under that role's register budget.
     if (warp >= 8) ptx::setmaxnreg_dec<kControlRegs>();
     if (warp == kProducerWarp) {
-        if (lane == 0) {
+        // The whole warp runs the schedule (its values stay warp-uniform);
+        // lane 0 issues the copies.
+        const uint32_t lead = lane == 0;
+        if (lead) {
             ptx::prefetch_tmap(&p.tm_q);
             ptx::prefetch_tmap(&p.tm_k);
             ptx::prefetch_tmap(&p.tm_v);
@@ -174,118 +184,145 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                 ptx::prefetch_tmap(&p.tm_kd);
                 ptx::prefetch_tmap(&p.tm_vd);
             }
-            ptx::mbar_arrive_expect_tx(&bars->q_full, 2 * kTileBytes);
-            for (int i = 0; i < 2; ++i)
-                for (int hf = 0; hf < 2; ++hf)
-                    ptx::tma_load_4d(sQ + i * kTileBytes + hf * kHalfBytes, &p.tm_q, &bars->q_full,
-                                     hf * 64, kvh * p.G, t0 + i * n, b);
-            int seq = 0;
-            bool ok = true;
-            for (int x = 0; x < n_items && ok; ++x) {
-                for (int kv = 0; kv < 2; ++kv, ++seq) {
-                    const int st = seq % kStages;
-                    const uint32_t ph = (seq / kStages) & 1;
-                    if (!ptx::mbar_wait(&bars->empty[st], ph ^ 1, wait_limit, abort_flag)) {
-                        flag_timeout(p, bars);
-                        ok = false;
-                        break;
-                    }
-                    ptx::mbar_arrive_expect_tx(&bars->full[st], kTileBytes);
-                    uint8_t* dst = sRing + st * kTileBytes;
-                    for (int hf = 0; hf < 2; ++hf) {
-                        if (x < n_seq) {
-                            ptx::tma_load_4d(dst + hf * kHalfBytes, kv ? &p.tm_v : &p.tm_k, &bars->full[st],
-                                             hf * 64, kvh, x * kBN, b);
-                        } else {
-                            const int row = t0 * p.Ld + (x - n_seq) * kBN;
-                            const CUtensorMap* m = kv ? &p.tm_vd : &p.tm_kd;
-                            if (p.depth_packed)
-                                ptx::tma_load_4d(dst + hf * kHalfBytes, m, &bars->full[st], hf * 64, row, kvh, b);
-                            else
-                                ptx::tma_load_4d(dst + hf * kHalfBytes, m, &bars->full[st], hf * 64, kvh, row, b);
-                        }
+        }
+        ptx::mbar_arrive_expect_tx_lead(&bars->q_full, 2 * kTileBytes, lead);
+        for (int i = 0; i < 2; ++i)
+            for (int hf = 0; hf < 2; ++hf)
+                ptx::tma_load_4d_lead(sQ + i * kTileBytes + hf * kHalfBytes, &p.tm_q, &bars->q_full, hf * 64,
+                                      kvh * p.G, t0 + i * n, b, lead);
+        int seq = 0;
+        bool ok = true;
+        for (int x = 0; x < n_items && ok; ++x) {
+            for (int kv = 0; kv < 2; ++kv, ++seq) {
+                const int st = seq % kStages;
+                const uint32_t ph = (seq / kStages) & 1;
+                if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->empty[st], ph ^ 1, wait_limit, abort_flag))) {
+                    if (lead) flag_timeout(p, bars);
+                    ok = false;
+                    break;
+                }
+                ptx::mbar_arrive_expect_tx_lead(&bars->full[st], kTileBytes, lead);
+                uint8_t* dst = sRing + st * kTileBytes;
+                for (int hf = 0; hf < 2; ++hf) {
+                    if (x < n_seq) {
+                        ptx::tma_load_4d_lead(dst + hf * kHalfBytes, kv ? &p.tm_v : &p.tm_k, &bars->full[st], hf * 64,
+                                              kvh, x * kBN, b, lead);
+                    } else {
+                        const int row = t0 * p.Ld + (x - n_seq) * kBN;
+                        const CUtensorMap* m = kv ? &p.tm_vd : &p.tm_kd;
+                        if (p.depth_packed)
+                            ptx::tma_load_4d_lead(dst + hf * kHalfBytes, m, &bars->full[st], hf * 64, row, kvh, b, lead);
+                        else
+                            ptx::tma_load_4d_lead(dst + hf * kHalfBytes, m, &bars->full[st], hf * 64, kvh, row, b, lead);
                     }
                 }
             }
-            // Drain: every load this CTA issued lands before the CTA can exit.
-            ptx::mbar_wait(&bars->q_full, 0, kNoPollLimit, nullptr);
-            for (int s = (seq > kStages ? seq - kStages : 0); s < seq; ++s)
-                ptx::mbar_wait(&bars->full[s % kStages], (s / kStages) & 1, kNoPollLimit, nullptr);
         }
+        // Drain: every load this CTA issued lands before the CTA can exit.
+        ptx::mbar_wait(&bars->q_full, 0, kNoPollLimit, nullptr);
+        for (int s = (seq > kStages ? seq - kStages : 0); s < seq; ++s)
+            ptx::mbar_wait(&bars->full[s % kStages], (s / kStages) & 1, kNoPollLimit, nullptr);
         __syncwarp();
     } else if (warp == kMmaWarp) {
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(kBM, kBN, 0, 0);
-            constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, 0, 1);
-            const uint32_t sQa = ptx::smem_u32(sQ);
-            const uint32_t sRa = ptx::smem_u32(sRing);
-            bool ok = ptx::mbar_wait(&bars->q_full, 0, wait_limit, abort_flag);
-            int cnt_p[2] = {0, 0};
-            auto part = [&](int i, int x) { return x < n_kv[i] || x >= n_seq; };
-            auto wait_full = [&](int seq) {
-                if (!ok) return;
-                if (!ptx::mbar_wait(&bars->full[seq % kStages], (seq / kStages) & 1, wait_limit, abort_flag)) {
-                    flag_timeout(p, bars);
-                    ok = false;
-                }
-                ptx::tc_fence_after();
-            };
-            auto issue_s = [&](int i, int seq) {
-                const uint32_t kt = sRa + (seq % kStages) * kTileBytes;
-                const uint32_t qt = sQa + i * kTileBytes;
-#pragma unroll
-                for (int k = 0; k < kD / 16; ++k)
-                    ptx::mma_ss(tmem + i * 128, desc_kmajor(qt, k), desc_kmajor(kt, k), idesc_qk, k > 0);
-                ptx::mma_commit(&bars->s_full[i]);
-            };
-            if (ok) ptx::tc_fence_after();
-            wait_full(0);
-            if (ok) {
-                for (int i = 0; i < 2; ++i)
-                    if (part(i, 0)) issue_s(i, 0);
-                ptx::mma_commit(&bars->empty[0]);
+        // The whole warp runs the schedule so that descriptors stay
+        // warp-uniform; lane 0 issues every MMA and commit. Descriptors are
+        // formed once per tile; a K step only adds a constant to the 14-bit
+        // address field (K-major: 32 B per 16 columns within a 128-byte row,
+        // 16 KB per 64-column half; MN-major: 16 rows of 128 B = 2048 B).
+        const uint32_t lead = lane == 0;
+        constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(kBM, kBN, 0, 0);
+        constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, 0, 1);
+        const uint32_t sQa = ptx::smem_u32(sQ);
+        const uint32_t sRa = ptx::smem_u32(sRing);
+        uint64_t dq_desc[2];
+        for (int i = 0; i < 2; ++i) dq_desc[i] = ptx::umma_desc_sw128(sQa + i * kTileBytes, 16, 1024);
+        auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, wait_limit, abort_flag));
+        };
+        bool ok = wait_all(&bars->q_full, 0);
+        if (!ok && lead) flag_timeout(p, bars);
+        ptx::tc_fence_after();
+        int cnt_p0 = 0, cnt_p1 = 0;
+        // S_i = Q_i K^T for the K tile in ring slot `seq`
+#define MODA_ISSUE_S(I, SEQ)                                                                   \
+    do {                                                                                       \
+        const uint64_t kd_ = ptx::umma_desc_sw128(sRa + ((SEQ) % kStages) * kTileBytes, 16, 1024); \
+        const uint64_t qd_ = dq_desc[I];                                                       \
+        _Pragma("unroll") for (int k = 0; k < kD / 16; ++k) {                                  \
+            const uint64_t off = (uint64_t)((k >> 2) * (kHalfBytes >> 4) + (k & 3) * 2);        \
+            ptx::mma_ss_lead(tmem + (I) * 128, qd_ + off, kd_ + off, idesc_qk, k > 0, lead);   \
+        }                                                                                      \
+        ptx::mma_commit_lead(&bars->s_full[I], lead);                                          \
+    } while (0)
+        if (ok) ok = wait_all(&bars->full[0], 0);
+        if (!ok && lead) flag_timeout(p, bars);
+        ptx::tc_fence_after();
+        if (ok) {
+            if (part(0, 0)) MODA_ISSUE_S(0, 0);
+            if (part(1, 0)) MODA_ISSUE_S(1, 0);
+            ptx::mma_commit_lead(&bars->empty[0], lead);
+        }
+        for (int x = 0; x < n_items && ok; ++x) {
+            const int sv = 2 * x + 1, sk = 2 * x + 2;
+            const bool next = x + 1 < n_items;
+            ok = wait_all(&bars->full[sv % kStages], (sv / kStages) & 1);
+            if (!ok) {
+                if (lead) flag_timeout(p, bars);
+                break;
             }
-            for (int x = 0; x < n_items && ok; ++x) {
-                const int sv = 2 * x + 1, sk = 2 * x + 2;
-                const bool next = x + 1 < n_items;
-                wait_full(sv);
-                bool k_ready = false;
-                for (int i = 0; i < 2 && ok; ++i) {
-                    if (part(i, x)) {
-                        if (!ptx::mbar_wait(&bars->p_full[i], cnt_p[i] & 1, wait_limit, abort_flag)) {
-                            flag_timeout(p, bars);
+            ptx::tc_fence_after();
+            const uint64_t vd = ptx::umma_desc_sw128(sRa + (sv % kStages) * kTileBytes, kHalfBytes, 1024);
+            bool k_ready = false;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                if (!ok) break;
+                if (part(i, x)) {
+                    // O_i += P_i V, fed chunk by chunk as the softmax
+                    // publishes P (32 keys per chunk = 2 MMA K-steps).
+                    const int cnt = i ? cnt_p1 : cnt_p0;
+#pragma unroll
+                    for (int c = 0; c < kPChunks; ++c) {
+                        if (!wait_all(&bars->p_full[i][c], cnt & 1)) {
+                            if (lead) flag_timeout(p, bars);
                             ok = false;
                             break;
                         }
                         ptx::tc_fence_after();
-                        const uint32_t vt = sRa + (sv % kStages) * kTileBytes;
 #pragma unroll
-                        for (int k = 0; k < kBN / 16; ++k)
-                            ptx::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8, desc_mnmajor(vt, k),
-                                        idesc_pv, (cnt_p[i] > 0 || k > 0) ? 1u : 0u);
-                        ++cnt_p[i];
-                    }
-                    if (next && part(i, x + 1)) {
-                        if (!k_ready) {
-                            wait_full(sk);
-                            k_ready = true;
-                            if (!ok) break;
+                        for (int kk = 0; kk < 8 / kPChunks; ++kk) {
+                            const int k = (8 / kPChunks) * c + kk;
+                            ptx::mma_ts_lead(tmem + 256 + i * 128, tmem + i * 128 + k * 8, vd + (uint64_t)(k * 128),
+                                             idesc_pv, (cnt > 0 || k > 0) ? 1u : 0u, lead);
                         }
-                        issue_s(i, sk);
                     }
+                    if (!ok) break;
+                    if (i) ++cnt_p1; else ++cnt_p0;
                 }
-                if (!ok) break;
-                ptx::mma_commit(&bars->empty[sv % kStages]);
-                if (next) ptx::mma_commit(&bars->empty[sk % kStages]);
+                if (next && part(i, x + 1)) {
+                    if (!k_ready) {
+                        if (!wait_all(&bars->full[sk % kStages], (sk / kStages) & 1)) {
+                            if (lead) flag_timeout(p, bars);
+                            ok = false;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        k_ready = true;
+                    }
+                    MODA_ISSUE_S(i, sk);
+                }
             }
-            if (ok) {
-                ptx::mma_commit(&bars->o_final[0]);
-                ptx::mma_commit(&bars->o_final[1]);
-            }
-            // Drain: all MMAs issued by this thread complete before TMEM is freed.
-            ptx::mma_commit(&bars->drain);
-            ptx::mbar_wait(&bars->drain, 0, kNoPollLimit, nullptr);
+            if (!ok) break;
+            ptx::mma_commit_lead(&bars->empty[sv % kStages], lead);
+            if (next) ptx::mma_commit_lead(&bars->empty[sk % kStages], lead);
         }
+#undef MODA_ISSUE_S
+        if (ok) {
+            ptx::mma_commit_lead(&bars->o_final[0], lead);
+            ptx::mma_commit_lead(&bars->o_final[1], lead);
+        }
+        // Drain: all MMAs issued by this warp complete before TMEM is freed.
+        ptx::mma_commit_lead(&bars->drain, lead);
+        ptx::mbar_wait(&bars->drain, 0, kNoPollLimit, nullptr);
         __syncwarp();
     } else if (warp < 8) {
         // ------------------------------------------------ softmax warpgroups
@@ -300,10 +337,10 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
         const int h = kvh * p.G + r % p.G;
         const float sl2 = p.sl2;
         float m = -INFINITY, l = 0.f;
-        const int n_it = n_kv[i] + n_dep;
         bool ok = true;
-        for (int it = 0; it < n_it; ++it) {
-            const int x = it < n_kv[i] ? it : it + (n_seq - n_kv[i]);
+        int it = 0;                        // items this tile has taken part in
+        for (int x = 0; x < n_items; ++x) {
+            if (!part(i, x)) continue;
             // tcgen05.ld / st below are warp-collective: every decision that
             // guards them is made warp-uniform.
             const bool got = ptx::mbar_wait(&bars->s_full[i], it & 1, wait_limit, abort_flag);
@@ -331,6 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                         if (kbase + c > t) s[c] = -INFINITY;
                 }
             } else {
+                // same-token mask: this row's depth rows are [tl*Ld, (tl+1)*Ld)
+                // of the unit's depth range
                 const int lo = tl * p.Ld - (x - n_seq) * kBN;
                 const int hi = lo + p.Ld;
 #pragma unroll
@@ -341,11 +380,15 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
             {
                 float mp[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) mp[e] = s[e];
+                for (int e = 0; e < 8; ++e) mp[e] = ptx::max3(s[e], s[8 + e], s[16 + e]);
 #pragma unroll
-                for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
-                mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                           fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+                for (int c = 24; c < 120; c += 16)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mp[e] = ptx::max3(mp[e], s[c + e], s[c + 8 + e]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mp[e] = fmaxf(mp[e], s[120 + e]);
+                mx = ptx::max3(ptx::max3(mp[0], mp[1], mp[2]), ptx::max3(mp[3], mp[4], mp[5]),
+                               fmaxf(mp[6], mp[7]));
             }
             const float mxs = mx * sl2;
             if (__any_sync(0xffffffffu, mxs > m + kRescaleThreshold)) {
@@ -369,34 +412,44 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                 l *= corr;
                 m = mnew;
             }
-            uint32_t pk[64];
             const float mref = (m == -INFINITY) ? 0.f : m;
             const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(-mref, -mref);
             float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                              make_float2(0.f, 0.f)};
+            // P in kPChunks chunks of 32 keys: each chunk goes to TMEM and is
+            // published at once, so the PV MMA starts on it while later
+            // chunks are still being exponentiated.
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const float2 xv = ptx::fma2(make_float2(s[2 * c], s[2 * c + 1]), sl2x2, nm2);
-                float2 pv;
-                if ((c & 7) >= kPolyFrom) {
-                    pv = ptx::exp2_poly2(xv);  // FMA pipe
-                } else {
-                    pv.x = ptx::ex2(xv.x);     // MUFU
-                    pv.y = ptx::ex2(xv.y);
+            for (int ch = 0; ch < kPChunks; ++ch) {
+                constexpr int kPairs = 64 / kPChunks;  // packed columns per chunk
+                uint32_t pk[kPairs];
+#pragma unroll
+                for (int e = 0; e < kPairs; ++e) {
+                    const int c = ch * kPairs + e;
+                    const float2 xv = ptx::fma2(make_float2(s[2 * c], s[2 * c + 1]), sl2x2, nm2);
+                    float2 pv;
+                    if ((c & 7) >= kPolyFrom) {
+                        pv = ptx::exp2_poly2(xv);  // FMA pipe
+                    } else {
+                        pv.x = ptx::ex2(xv.x);     // MUFU
+                        pv.y = ptx::ex2(xv.y);
+                    }
+                    acc[c & 3] = ptx::add2(acc[c & 3], pv);
+                    pk[e] = ptx::pack_bf16x2(pv.x, pv.y);
                 }
-                acc[c & 3] = ptx::add2(acc[c & 3], pv);
-                pk[c] = ptx::pack_bf16x2(pv.x, pv.y);
+#pragma unroll
+                for (int q = 0; q < kPairs / 16; ++q)
+                    ptx::tmem_st16(tS + ch * kPairs + q * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[q * 16]));
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&bars->p_full[i][ch]);
             }
             {
                 const float2 a01 = ptx::add2(acc[0], acc[1]), a23 = ptx::add2(acc[2], acc[3]);
                 const float2 a = ptx::add2(a01, a23);
                 l += a.x + a.y;
             }
-            ptx::tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
-            ptx::tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
-            ptx::tmem_wait_st();
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&bars->p_full[i]);
+            ++it;
         }
         if (ok) {
             const bool got = ptx::mbar_wait(&bars->o_final[i], 0, wait_limit, abort_flag);
