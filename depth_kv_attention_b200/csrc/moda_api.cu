@@ -83,12 +83,12 @@ moda_status run_fwd(FwdArgs& a, void* stream, moda_impl impl) {
 }
 
 // Workspace: [fp32 D, B*Hq*T, rounded to 256 B] then, for bf16 (tensor-core
-// path), the fp32 accumulators of dq [B,T,Hq,d], dk and dv [B,T,Hkv,d].
+// path), the fp32 accumulators of dk and dv [B,T,Hkv,d].
 size_t bwd_ws_rowD_bytes(int B, int T, int Hq) {
     return ((size_t)B * Hq * T * sizeof(float) + 255) & ~size_t(255);
 }
 size_t bwd_ws_bytes(int B, int T, int Hq, int Hkv, int d, bool with_acc) {
-    size_t acc = with_acc ? (size_t)B * T * (Hq + 2 * Hkv) * d * sizeof(float) : 0;
+    size_t acc = with_acc ? (size_t)B * T * 2 * Hkv * d * sizeof(float) : 0;
     return bwd_ws_rowD_bytes(B, T, Hq) + acc;
 }
 
@@ -165,8 +165,7 @@ moda_status moda_bwd_ex(const void* q, const void* k, const void* v, const void*
     a.rowD = static_cast<float*>(workspace);
     if (dtype == MODA_BF16) {
         char* base = static_cast<char*>(workspace) + bwd_ws_rowD_bytes(B, T, Hq);
-        a.dq_acc = reinterpret_cast<float*>(base);
-        a.dk_acc = a.dq_acc + (size_t)B * T * Hq * d;
+        a.dk_acc = reinterpret_cast<float*>(base);
         a.dv_acc = a.dk_acc + (size_t)B * T * Hkv * d;
     }
     cudaError_t e = status_ptr(&a.f.status, &a.f.wait_limit);

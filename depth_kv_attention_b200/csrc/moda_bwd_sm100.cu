@@ -10,26 +10,21 @@
 //
 // Launch sequence (one stream):
 //   1. D = rowsum(dout * out)                      (SIMT, shared with the SIMT path)
-//   2. dq_acc = scale * sum_i dS'_i kd_i            (SIMT; plain store, 0 when Ld = 0)
-//   3. dkd, dvd                                     (SIMT, shared with the SIMT path)
-//   4. sequence part, KV-major, tensor cores        (this file): dq, dk and dv
-//      partials added into fp32 accumulators with vector fp32 reductions
-//   5. dq, dk, dv = bf16(accumulators)
+//   2. dkd, dvd                                     (SIMT, shared with the SIMT path)
+//   3. dk, dv: KV-major tensor-core kernel; partial sums of a key tile over a
+//      chunk of query tiles go to fp32 accumulators with vector reductions
+//   4. dq: query-major tensor-core kernel over the causal key tiles and the
+//      query tile's own depth chunks; dq accumulates in TMEM and is written
+//      once, in bf16 (no dq reductions between CTAs)
+//   5. dk, dv = bf16(accumulators)
+// Splitting dq from dk/dv recomputes S and dP once more (7 instead of 5
+// GEMMs per tile pair) but removes the per-pair fp32 dq reductions, which for
+// wide GQA (G = 32, 4 tokens per 128-row tile) would move gigabytes through L2.
 //
-// Kernel 4: one CTA per (b, kv-head, 128-key tile, chunk of query tiles); it
-// walks its share of the query tiles of the rows that can see its keys
-// (tokens t >= j0), 128 rows each in the
-// forward's token-major GQA order (n = 128 / G tokens x G heads), so the
-// G heads' contributions to dk / dv sum inside the TMEM accumulators.
-// Per query tile:
-//   S^T  = K Q^T   and   dP^T = V dO^T          (SS MMAs -> TMEM)
-//   CUDA cores (one thread per key): P^T, dS^T -> bf16 -> TMEM (over S^T and
-//   dP^T) for the next two MMAs, and dS -> shared memory for the third
-//   dV += P^T dO,  dK += dS^T Q                  (A operand from TMEM)
-//   dQ_tile = dS K                               (A from shared memory) -> TMEM
-//   CUDA cores (one thread per query row): red.global.add.v4.f32 into dq_acc.
-// TMEM: S^T | dP^T | dV | dK (128 fp32 columns each); dQ_tile reuses S^T's
-// columns once dV has read P^T (tcgen05.mma of one thread run in order).
+// Both kernels put query rows in the forward's token-major GQA order (a
+// 128-row tile = n = 128/G tokens x G heads), one warp issues the TMA loads
+// and one the MMAs (whole-warp control, one lane issues), four warps do the
+// elementwise work with one thread per TMEM lane.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -43,8 +38,7 @@ namespace moda {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kBK = 128;          // keys per CTA
-constexpr int kStages = 2;        // query-tile ring (Q and dO per stage)
+constexpr int kBK = 128;          // keys per key tile
 constexpr int kTile = 128 * kD * 2;
 constexpr int kHalf = kTile / 2;
 constexpr int kThreads = 192;     // warps 0-3 compute, 4 TMA producer, 5 MMA
@@ -52,39 +46,12 @@ constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr float kLog2e = 1.4426950408889634f;
 
-struct TcBwdParams {
-    CUtensorMap tm_q, tm_do, tm_k, tm_v;
-    const float* lse;
-    const float* rowD;
-    float* dq_acc;
-    float* dk_acc;  // [B,T,Hkv,d] fp32, zeroed before the launch
-    float* dv_acc;
-    int B, T, Hq, Hkv, G, n, nkt, qchunk;
-    float sl2, scale;
-    unsigned int* status;
-    unsigned int wait_limit;
-};
-
-struct __align__(8) Bars {
-    uint64_t kv_full;
-    uint64_t qd_full[kStages];
-    uint64_t qd_empty[kStages];
-    uint64_t s_full, p_full, dq_full, tmem_free, fin, drain;
-    uint32_t tmem_base;
-    int abort_flag;
-};
-
-// K, V, ring of (Q, dO), dS, then the tile's lse / D and the barriers.
-constexpr int kSmemBytes = 2 * kTile + kStages * 2 * kTile + kTile + 2 * 128 * 4 + 128 + 1024;
-static_assert(sizeof(Bars) <= 128, "barrier block");
-static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-
-__device__ __forceinline__ uint64_t desc_k(uint32_t tile, int k16) {
-    return ptx::umma_desc_sw128(tile + (k16 >> 2) * kHalf + (k16 & 3) * 32, 16, 1024);
-}
-__device__ __forceinline__ uint64_t desc_mn(uint32_t tile, int k16) {
-    return ptx::umma_desc_sw128(tile + k16 * 16 * 128, kHalf, 1024);
-}
+__device__ __forceinline__ uint64_t kdesc(uint32_t tile) { return ptx::umma_desc_sw128(tile, 16, 1024); }
+__device__ __forceinline__ uint64_t mndesc(uint32_t tile) { return ptx::umma_desc_sw128(tile, kHalf, 1024); }
+// K step k of a K-major tile: 32 B within the 128-byte row, 16 KB per half.
+__device__ __forceinline__ uint64_t koff(int k) { return (uint64_t)((k >> 2) * (kHalf >> 4) + (k & 3) * 2); }
+// K step k of an MN-major tile: 16 rows of 128 B.
+__device__ __forceinline__ uint64_t mnoff(int k) { return (uint64_t)(k * 128); }
 
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
@@ -110,58 +77,84 @@ __device__ __forceinline__ bool all_compute(bool v) {
     return r != 0;
 }
 
-__device__ __forceinline__ void flag_timeout(TcBwdParams const& p, Bars* bars) {
+struct __align__(8) Bars {
+    uint64_t kv_full;            // dk/dv kernel: K, V tile | dq kernel: Q, dO tile
+    uint64_t full[4];            // ring slots
+    uint64_t empty[4];
+    uint64_t s_full, dp_full, p_full, fin, drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__device__ __forceinline__ void flag_timeout(unsigned int* status, Bars* bars) {
     *reinterpret_cast<volatile int*>(&bars->abort_flag) = 1;
-    atomicOr(p.status, 1u);
+    atomicOr(status, 1u);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) moda_bwd_seq_tc_kernel(const __grid_constant__ TcBwdParams p) {
+__device__ __forceinline__ void init_bars(Bars* bars, int stages) {
+    ptx::mbar_init(&bars->kv_full, 1);
+    for (int s = 0; s < stages; ++s) {
+        ptx::mbar_init(&bars->full[s], 1);
+        ptx::mbar_init(&bars->empty[s], 1);
+    }
+    ptx::mbar_init(&bars->s_full, 1);
+    ptx::mbar_init(&bars->dp_full, 1);
+    ptx::mbar_init(&bars->p_full, 128);
+    ptx::mbar_init(&bars->fin, 1);
+    ptx::mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    ptx::fence_barrier_init();
+    ptx::fence_proxy_async_smem();
+}
+
+// ===================================================================== dk, dv
+struct DkvParams {
+    CUtensorMap tm_q, tm_do, tm_k, tm_v;
+    const float* lse;
+    const float* rowD;
+    float* dk_acc;  // [B,T,Hkv,d] fp32, zeroed before the launch
+    float* dv_acc;
+    int B, T, Hq, Hkv, G, n, gshift, qchunk;
+    float sl2, scale;
+    unsigned int* status;
+    unsigned int wait_limit;
+};
+constexpr int kDkvStages = 2;  // ring of (Q, dO) pairs
+constexpr int kDkvSmem = 2 * kTile + kDkvStages * 2 * kTile + 2 * 128 * 4 + 256 + 1024;
+static_assert(kDkvSmem <= 232448, "shared memory per CTA");
+static_assert(sizeof(Bars) <= 256, "barrier block");
+
+// One CTA per (key tile = blockIdx.x, chunk of query tokens = blockIdx.y,
+// (b, kv-head) = blockIdx.z). TMEM: S^T | dP^T | dV | dK, 128 columns each.
+// Per query tile: S^T = K Q^T, dP^T = V dO^T; the compute warps (thread =
+// key) form P^T and dS^T in bf16 over S^T / dP^T; dV += P^T dO and
+// dK += dS^T Q take them as TMEM A operands. The next tile's S^T / dP^T
+// follow those two MMAs in issue order, so they overwrite P^T / dS^T only
+// after they are read.
+__global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid_constant__ DkvParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sK = smem;
     uint8_t* sV = smem + kTile;
-    uint8_t* sRing = smem + 2 * kTile;                  // stage s: Q at +2s*kTile, dO at +(2s+1)*kTile
-    uint8_t* sDS = sRing + kStages * 2 * kTile;
-    float* sStat = reinterpret_cast<float*>(sDS + kTile);  // [lse2 128 | D 128] of the query tile
+    uint8_t* sRing = smem + 2 * kTile;  // stage s: Q at +2s*kTile, dO at +(2s+1)*kTile
+    float* sStat = reinterpret_cast<float*>(sRing + kDkvStages * 2 * kTile);  // [lse2 | D] of the query tile
     Bars* bars = reinterpret_cast<Bars*>(sStat + 256);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const uint32_t wait_limit = p.wait_limit;
     volatile int* abort_flag = &bars->abort_flag;
-
-    // Work item: key tile = blockIdx.x (fastest), chunk of query tokens =
-    // blockIdx.y, (b, kv-head) = blockIdx.z. A chunk is qchunk query tiles of
-    // absolute token range [c*qchunk*n, (c+1)*qchunk*n); the CTAs in flight
-    // at one time are the key tiles of one or two chunks, so their fp32 dq
-    // reductions land on the same few MB of dq rows (L2-resident). Key tiles
-    // that no row of the chunk can see exit at once.
     const int b = blockIdx.z / p.Hkv, kvh = blockIdx.z % p.Hkv;
-    const int kt = blockIdx.x;
-    const int j0 = kt * kBK;
+    const int j0 = blockIdx.x * kBK;
     const int n = p.n;
-    const int c_lo = blockIdx.y * p.qchunk * n;                      // first token of the chunk
-    const int c_hi = min(p.T, (blockIdx.y + 1) * p.qchunk * n);      // one past its last token
-    const int t_first = max(j0, c_lo);                               // multiple of n
+    // A chunk is qchunk query tiles of absolute tokens [c*qchunk*n, ...); the
+    // CTAs in flight at once cover one or two chunks. Key tiles that no row of
+    // the chunk can see exit at once.
+    const int c_lo = blockIdx.y * p.qchunk * n;
+    const int c_hi = min(p.T, (blockIdx.y + 1) * p.qchunk * n);
+    const int t_first = max(j0, c_lo);  // a multiple of n
     if (t_first >= c_hi) return;
     const int nq = (c_hi - t_first + n - 1) / n;
-    const int q_first = (t_first - j0) / n;                          // query tiles counted from j0
 
-    if (threadIdx.x == 0) {
-        ptx::mbar_init(&bars->kv_full, 1);
-        for (int s = 0; s < kStages; ++s) {
-            ptx::mbar_init(&bars->qd_full[s], 1);
-            ptx::mbar_init(&bars->qd_empty[s], 1);
-        }
-        ptx::mbar_init(&bars->s_full, 1);
-        ptx::mbar_init(&bars->p_full, 128);
-        ptx::mbar_init(&bars->dq_full, 1);
-        ptx::mbar_init(&bars->tmem_free, 128);
-        ptx::mbar_init(&bars->fin, 1);
-        ptx::mbar_init(&bars->drain, 1);
-        bars->abort_flag = 0;
-        ptx::fence_barrier_init();
-        ptx::fence_proxy_async_smem();
-    }
+    if (threadIdx.x == 0) init_bars(bars, kDkvStages);
     if (warp == 0) {
         ptx::tmem_alloc(&bars->tmem_base, 512);
         ptx::tmem_relinquish();
@@ -170,105 +163,98 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_seq_tc_kernel(const __gr
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, p.wait_limit, abort_flag));
+    };
 
     if (warp == kProducerWarp) {
-        if (lane == 0) {
+        const uint32_t lead = lane == 0;
+        if (lead) {
             ptx::prefetch_tmap(&p.tm_q);
             ptx::prefetch_tmap(&p.tm_do);
             ptx::prefetch_tmap(&p.tm_k);
             ptx::prefetch_tmap(&p.tm_v);
-            ptx::mbar_arrive_expect_tx(&bars->kv_full, 2 * kTile);
-            for (int hf = 0; hf < 2; ++hf) {
-                ptx::tma_load_4d(sK + hf * kHalf, &p.tm_k, &bars->kv_full, hf * 64, kvh, j0, b);
-                ptx::tma_load_4d(sV + hf * kHalf, &p.tm_v, &bars->kv_full, hf * 64, kvh, j0, b);
-            }
-            int issued = 0;
-            for (int i = 0; i < nq; ++i) {
-                const int st = i % kStages;
-                const uint32_t ph = (i / kStages) & 1;
-                if (!ptx::mbar_wait(&bars->qd_empty[st], ph ^ 1, wait_limit, abort_flag)) {
-                    flag_timeout(p, bars);
-                    break;
-                }
-                ptx::mbar_arrive_expect_tx(&bars->qd_full[st], 2 * kTile);
-                uint8_t* q_dst = sRing + (2 * st) * kTile;
-                uint8_t* do_dst = sRing + (2 * st + 1) * kTile;
-                const int tq0 = j0 + (q_first + i) * n;
-                for (int hf = 0; hf < 2; ++hf) {
-                    ptx::tma_load_4d(q_dst + hf * kHalf, &p.tm_q, &bars->qd_full[st], hf * 64, kvh * p.G, tq0, b);
-                    ptx::tma_load_4d(do_dst + hf * kHalf, &p.tm_do, &bars->qd_full[st], hf * 64, kvh * p.G, tq0, b);
-                }
-                issued = i + 1;
-            }
-            // Drain: every load issued lands before the CTA exits.
-            ptx::mbar_wait(&bars->kv_full, 0, 0, nullptr);
-            for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-                ptx::mbar_wait(&bars->qd_full[i % kStages], (i / kStages) & 1, 0, nullptr);
         }
+        ptx::mbar_arrive_expect_tx_lead(&bars->kv_full, 2 * kTile, lead);
+        for (int hf = 0; hf < 2; ++hf) {
+            ptx::tma_load_4d_lead(sK + hf * kHalf, &p.tm_k, &bars->kv_full, hf * 64, kvh, j0, b, lead);
+            ptx::tma_load_4d_lead(sV + hf * kHalf, &p.tm_v, &bars->kv_full, hf * 64, kvh, j0, b, lead);
+        }
+        int issued = 0;
+        for (int i = 0; i < nq; ++i) {
+            const int st = i % kDkvStages;
+            if (!wait_all(&bars->empty[st], ((i / kDkvStages) & 1) ^ 1)) {
+                if (lead) flag_timeout(p.status, bars);
+                break;
+            }
+            ptx::mbar_arrive_expect_tx_lead(&bars->full[st], 2 * kTile, lead);
+            const int tq0 = t_first + i * n;
+            for (int hf = 0; hf < 2; ++hf) {
+                ptx::tma_load_4d_lead(sRing + (2 * st) * kTile + hf * kHalf, &p.tm_q, &bars->full[st], hf * 64,
+                                      kvh * p.G, tq0, b, lead);
+                ptx::tma_load_4d_lead(sRing + (2 * st + 1) * kTile + hf * kHalf, &p.tm_do, &bars->full[st],
+                                      hf * 64, kvh * p.G, tq0, b, lead);
+            }
+            issued = i + 1;
+        }
+        ptx::mbar_wait(&bars->kv_full, 0, 0, nullptr);
+        for (int i = (issued > kDkvStages ? issued - kDkvStages : 0); i < issued; ++i)
+            ptx::mbar_wait(&bars->full[i % kDkvStages], (i / kDkvStages) & 1, 0, nullptr);
         __syncwarp();
     } else if (warp == kMmaWarp) {
-        if (lane == 0) {
-            constexpr uint32_t idesc_ss = ptx::idesc_bf16_f32(128, 128, 0, 0);
-            constexpr uint32_t idesc_ts = ptx::idesc_bf16_f32(128, kD, 0, 1);
-            constexpr uint32_t idesc_dq = ptx::idesc_bf16_f32(128, kD, 1, 1);
-            const uint32_t aK = ptx::smem_u32(sK), aV = ptx::smem_u32(sV), aDS = ptx::smem_u32(sDS);
-            const uint32_t aRing = ptx::smem_u32(sRing);
-            bool ok = ptx::mbar_wait(&bars->kv_full, 0, wait_limit, abort_flag);
-            if (!ok) flag_timeout(p, bars);
-            ptx::tc_fence_after();
-            for (int i = 0; i < nq && ok; ++i) {
-                const int st = i % kStages;
-                const uint32_t aQ = aRing + (2 * st) * kTile, aDO = aRing + (2 * st + 1) * kTile;
-                ok = ptx::mbar_wait(&bars->qd_full[st], (i / kStages) & 1, wait_limit, abort_flag);
-                if (ok && i > 0) ok = ptx::mbar_wait(&bars->tmem_free, (i - 1) & 1, wait_limit, abort_flag);
-                if (!ok) {
-                    flag_timeout(p, bars);
-                    break;
-                }
-                ptx::tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < kD / 16; ++k)
-                    ptx::mma_ss(tmem + 0, desc_k(aK, k), desc_k(aQ, k), idesc_ss, k > 0);
-#pragma unroll
-                for (int k = 0; k < kD / 16; ++k)
-                    ptx::mma_ss(tmem + 128, desc_k(aV, k), desc_k(aDO, k), idesc_ss, k > 0);
-                ptx::mma_commit(&bars->s_full);
-                if (!ptx::mbar_wait(&bars->p_full, i & 1, wait_limit, abort_flag)) {
-                    flag_timeout(p, bars);
-                    ok = false;
-                    break;
-                }
-                ptx::tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < 128 / 16; ++k)
-                    ptx::mma_ts(tmem + 256, tmem + 0 + k * 8, desc_mn(aDO, k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-                for (int k = 0; k < 128 / 16; ++k)
-                    ptx::mma_ts(tmem + 384, tmem + 128 + k * 8, desc_mn(aQ, k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-                for (int k = 0; k < kBK / 16; ++k)
-                    ptx::mma_ss(tmem + 0, desc_mn(aDS, k), desc_mn(aK, k), idesc_dq, k > 0);
-                ptx::mma_commit(&bars->dq_full);
-                ptx::mma_commit(&bars->qd_empty[st]);
+        const uint32_t lead = lane == 0;
+        constexpr uint32_t idesc_ss = ptx::idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint32_t idesc_ts = ptx::idesc_bf16_f32(128, kD, 0, 1);
+        const uint64_t dK = kdesc(ptx::smem_u32(sK)), dV = kdesc(ptx::smem_u32(sV));
+        const uint32_t aRing = ptx::smem_u32(sRing);
+        bool ok = wait_all(&bars->kv_full, 0);
+        if (!ok && lead) flag_timeout(p.status, bars);
+        ptx::tc_fence_after();
+        for (int i = 0; i < nq && ok; ++i) {
+            const int st = i % kDkvStages;
+            const uint32_t aQ = aRing + (2 * st) * kTile, aDO = aRing + (2 * st + 1) * kTile;
+            ok = wait_all(&bars->full[st], (i / kDkvStages) & 1);
+            if (!ok) {
+                if (lead) flag_timeout(p.status, bars);
+                break;
             }
-            if (ok) ptx::mma_commit(&bars->fin);
-            ptx::mma_commit(&bars->drain);
-            ptx::mbar_wait(&bars->drain, 0, 0, nullptr);
+            ptx::tc_fence_after();
+            const uint64_t dQk = kdesc(aQ), dOk = kdesc(aDO), dQm = mndesc(aQ), dOm = mndesc(aDO);
+#pragma unroll
+            for (int k = 0; k < kD / 16; ++k) ptx::mma_ss_lead(tmem + 0, dK + koff(k), dQk + koff(k), idesc_ss, k > 0, lead);
+#pragma unroll
+            for (int k = 0; k < kD / 16; ++k) ptx::mma_ss_lead(tmem + 128, dV + koff(k), dOk + koff(k), idesc_ss, k > 0, lead);
+            ptx::mma_commit_lead(&bars->s_full, lead);
+            if (!wait_all(&bars->p_full, i & 1)) {
+                if (lead) flag_timeout(p.status, bars);
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 128 / 16; ++k)
+                ptx::mma_ts_lead(tmem + 256, tmem + 0 + k * 8, dOm + mnoff(k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u, lead);
+#pragma unroll
+            for (int k = 0; k < 128 / 16; ++k)
+                ptx::mma_ts_lead(tmem + 384, tmem + 128 + k * 8, dQm + mnoff(k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u, lead);
+            ptx::mma_commit_lead(&bars->empty[st], lead);
         }
+        if (ok) ptx::mma_commit_lead(&bars->fin, lead);
+        ptx::mma_commit_lead(&bars->drain, lead);
+        ptx::mbar_wait(&bars->drain, 0, 0, nullptr);
         __syncwarp();
     } else {
         // ------------------------------------------------------ compute warps
-        const int r = warp * 32 + lane;                 // TMEM lane
+        const int r = warp * 32 + lane;  // TMEM lane
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const int j = j0 + r;                           // this thread's key
+        const int j = j0 + r;            // this thread's key
         const float sl2 = p.sl2;
+        const int gshift = p.gshift;
         bool ok = true;
-        int gshift = 0;
-        while ((1 << gshift) < p.G) ++gshift;
-        // lse (log2 units) and D of row r of query tile i; loaded one tile
+        // lse (log2 units) and D of row r of query tile i, loaded one tile
         // ahead so the global-memory latency stays off the critical path.
         auto load_stat = [&](int i, float& l2, float& dd) {
-            const int t = j0 + (q_first + i) * n + (r >> gshift), h = kvh * p.G + (r & (p.G - 1));
+            const int t = t_first + i * n + (r >> gshift), h = kvh * p.G + (r & (p.G - 1));
             if (t < p.T) {
                 const long long ix = ((long long)b * p.Hq + h) * p.T + t;
                 l2 = p.lse[ix] * kLog2e;
@@ -281,22 +267,22 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_seq_tc_kernel(const __gr
         float nl2, nD;
         load_stat(0, nl2, nD);
         for (int i = 0; i < nq; ++i) {
-            const int tq0 = j0 + (q_first + i) * n;
+            const int tq0 = t_first + i * n;
             float* st_lse = sStat;
             float* st_D = sStat + 128;
             named_sync_compute();  // the previous tile's readers are done
             st_lse[r] = nl2;
             st_D[r] = nD;
             if (i + 1 < nq) load_stat(i + 1, nl2, nD);
-            const bool got = ptx::mbar_wait(&bars->s_full, i & 1, wait_limit, abort_flag);
+            const bool got = ptx::mbar_wait(&bars->s_full, i & 1, p.wait_limit, abort_flag);
             if (!all_compute(got)) {  // also publishes st_lse / st_D
-                flag_timeout(p, bars);
+                flag_timeout(p.status, bars);
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
-            // key j is visible to row rr iff j <= t(rr) = tq0 + (rr >> gshift),
-            // i.e. rows rr < (j - tq0) << gshift are masked.
+            // key j is visible to row rr iff j <= tq0 + (rr >> gshift): rows
+            // rr < (j - tq0) << gshift are masked.
             const int mask_below = j > tq0 ? (j - tq0) << gshift : 0;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
@@ -319,55 +305,19 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_seq_tc_kernel(const __gr
                     pp[e2] = ptx::pack_bf16x2(pv[0], pv[1]);
                     dd[e2] = ptx::pack_bf16x2(dv[0], dv[1]);
                 }
+                // chunk c's packed columns [16c, 16c+16) lie in columns this
+                // thread has already read
                 ptx::tmem_st16(tmem + lane_off + 0 + 16 * c, pp);
                 ptx::tmem_st16(tmem + lane_off + 128 + 16 * c, dd);
-                // dS into shared memory, [key][row] with rows contiguous (the
-                // MN-major A operand of dQ = dS K), 128-byte swizzle.
-                uint8_t* half = sDS + (c >> 1) * kHalf + r * 128;
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const int chunk = ((c & 1) * 4 + v) ^ (r & 7);
-                    *reinterpret_cast<uint4*>(half + chunk * 16) =
-                        make_uint4(dd[4 * v], dd[4 * v + 1], dd[4 * v + 2], dd[4 * v + 3]);
-                }
             }
             ptx::tmem_wait_st();
-            ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars->p_full);
-
-            // dQ tile (lane = query row) -> fp32 reductions into dq_acc.
-            const bool got2 = ptx::mbar_wait(&bars->dq_full, i & 1, wait_limit, abort_flag);
-            if (!all_compute(got2)) {
-                flag_timeout(p, bars);
-                ok = false;
-                break;
-            }
-            ptx::tc_fence_after();
-            {
-                const int t = tq0 + (r >> gshift), h = kvh * p.G + (r & (p.G - 1));
-                float* dst = p.dq_acc + (((long long)b * p.T + (t < p.T ? t : 0)) * p.Hq + h) * kD;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t o[32];
-                    ptx::tmem_ld32(tmem + lane_off + 32 * c, o);
-                    ptx::tmem_wait_ld();
-                    if (t < p.T) {
-#pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            red_add_v4(dst + 32 * c + 4 * v, __uint_as_float(o[4 * v]) * p.scale,
-                                       __uint_as_float(o[4 * v + 1]) * p.scale, __uint_as_float(o[4 * v + 2]) * p.scale,
-                                       __uint_as_float(o[4 * v + 3]) * p.scale);
-                    }
-                }
-            }
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&bars->tmem_free);
         }
         if (ok) {
-            const bool got = ptx::mbar_wait(&bars->fin, 0, wait_limit, abort_flag);
+            const bool got = ptx::mbar_wait(&bars->fin, 0, p.wait_limit, abort_flag);
             if (!all_compute(got)) {
-                flag_timeout(p, bars);
+                flag_timeout(p.status, bars);
                 ok = false;
             }
         }
@@ -406,75 +356,280 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_seq_tc_kernel(const __gr
     }
 }
 
-// dq_acc[row] = scale * sum_i dS'_i kd_i over the row's own depth entries (a
-// plain store that initialises the accumulator; zero when Ld = 0). Four
-// threads per query row, each owning 16 feature pairs.
-__global__ void __launch_bounds__(256) bwd_depth_dq_kernel(BwdArgs a) {
-    const FwdArgs& f = a.f;
-    constexpr int TPR = 4, NP = kD / (2 * TPR);
-    const long long rows = (long long)f.B * f.T * f.Hq;
-    const long long row = (long long)blockIdx.x * (blockDim.x / TPR) + threadIdx.x / TPR;
-    const int u = threadIdx.x % TPR;
-    const bool valid = row < rows;
-    const long long rc = valid ? row : rows - 1;
-    const int h = rc % f.Hq;
-    const int t = (rc / f.Hq) % f.T;
-    const int b = rc / ((long long)f.Hq * f.T);
-    const int kvh = h / f.G;
-    const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(f.q) + rc * kD;
-    const __nv_bfloat16* DO = static_cast<const __nv_bfloat16*>(a.dout) + rc * kD;
-    float2 q[NP], dO[NP], acc[NP];
-#pragma unroll
-    for (int i = 0; i < NP; ++i) {
-        const int c = 2 * (TPR * i + u);
-        q[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Q + c));
-        dO[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(DO + c));
-        acc[i] = make_float2(0.f, 0.f);
+// ========================================================================= dq
+struct DqParams {
+    CUtensorMap tm_q, tm_do, tm_k, tm_v, tm_kd, tm_vd;
+    const float* lse;
+    const float* rowD;
+    void* dq;  // [B,T,Hq,d] bf16
+    int B, T, Hq, Hkv, G, n, Ld, nqt;
+    float sl2, scale;
+    unsigned int* status;
+    unsigned int wait_limit;
+};
+constexpr int kDqStages = 4;  // ring of K / V tiles, one per slot
+constexpr int kDqSmem = 2 * kTile + kDqStages * kTile + 256 + 1024;
+static_assert(kDqSmem <= 232448, "shared memory per CTA");
+
+// One CTA per query tile (n tokens x G heads of one kv group), latest tokens
+// first. Items: the causal key tiles, then the tile's own depth chunks (rows
+// t0*Ld + 128*d .. of the [B, T*Ld, Hkv, d] view, same-token mask).
+// TMEM: R0 | R1 (S and dP alternate between them) | dQ. S(x) sits in
+// R[x % 2] and dP(x) in R[(x + 1) % 2]. Once the compute warps publish
+// dS(x) (written over S(x)), the MMA warp issues, in this order:
+//   S(x+1) = Q K(x+1)^T   into R[(x+1) % 2] (dP(x) there has been read)
+//   dQ    += dS(x) K(x)   A = dS(x) from R[x % 2]
+//   dP(x+1) = dO V(x+1)^T into R[x % 2], after dQ has read dS(x) there
+// so the compute warps exponentiate S(x+1) while dQ and dP(x+1) run, then
+// form dS(x+1) = P (dP - D).
+__global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_constant__ DqParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = smem;
+    uint8_t* sDO = smem + kTile;
+    uint8_t* sRing = smem + 2 * kTile;
+    Bars* bars = reinterpret_cast<Bars*>(sRing + kDqStages * kTile);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    volatile int* abort_flag = &bars->abort_flag;
+    const int bh = blockIdx.x % (p.B * p.Hkv);
+    const int qt = p.nqt - 1 - blockIdx.x / (p.B * p.Hkv);  // latest tokens (most keys) first
+    const int b = bh / p.Hkv, kvh = bh % p.Hkv;
+    const int n = p.n;
+    const int t0 = qt * n;
+    const int nv = min(n, p.T - t0);                   // tokens of the tile inside the sequence
+    const int n_kv = (t0 + nv - 1) / kBK + 1;
+    const int n_dep = (nv * p.Ld + kBK - 1) / kBK;
+    const int n_items = n_kv + n_dep;
+
+    if (threadIdx.x == 0) init_bars(bars, kDqStages);
+    if (warp == 0) {
+        ptx::tmem_alloc(&bars->tmem_base, 512);
+        ptx::tmem_relinquish();
     }
-    const long long rix = ((long long)b * f.Hq + h) * f.T + t;
-    const float lse2 = f.lse[rix] * kLog2e, Drow = a.rowD[rix], sl2 = f.scale * kLog2e;
-    for (int i = 0; i < f.Ld; ++i) {
-        const long long off = ((((long long)b * f.T + t) * f.Ld + i) * f.Hkv + kvh) * kD;
-        const __nv_bfloat16* KD = static_cast<const __nv_bfloat16*>(f.kd) + off;
-        const __nv_bfloat16* VD = static_cast<const __nv_bfloat16*>(f.vd) + off;
-        float2 kr[NP];
-        float s = 0.f, dp = 0.f;
-#pragma unroll
-        for (int e = 0; e < NP; ++e) {
-            const int c = 2 * (TPR * e + u);
-            kr[e] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(KD + c));
-            const float2 vr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(VD + c));
-            s = fmaf(q[e].x, kr[e].x, fmaf(q[e].y, kr[e].y, s));
-            dp = fmaf(dO[e].x, vr.x, fmaf(dO[e].y, vr.y, dp));
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, p.wait_limit, abort_flag));
+    };
+
+    if (warp == kProducerWarp) {
+        const uint32_t lead = lane == 0;
+        if (lead) {
+            ptx::prefetch_tmap(&p.tm_q);
+            ptx::prefetch_tmap(&p.tm_do);
+            ptx::prefetch_tmap(&p.tm_k);
+            ptx::prefetch_tmap(&p.tm_v);
+            if (p.Ld > 0) {
+                ptx::prefetch_tmap(&p.tm_kd);
+                ptx::prefetch_tmap(&p.tm_vd);
+            }
         }
-#pragma unroll
-        for (int o = 1; o < TPR; o <<= 1) {
-            s += __shfl_xor_sync(0xffffffffu, s, o);
-            dp += __shfl_xor_sync(0xffffffffu, dp, o);
+        ptx::mbar_arrive_expect_tx_lead(&bars->kv_full, 2 * kTile, lead);
+        for (int hf = 0; hf < 2; ++hf) {
+            ptx::tma_load_4d_lead(sQ + hf * kHalf, &p.tm_q, &bars->kv_full, hf * 64, kvh * p.G, t0, b, lead);
+            ptx::tma_load_4d_lead(sDO + hf * kHalf, &p.tm_do, &bars->kv_full, hf * 64, kvh * p.G, t0, b, lead);
         }
-        const float ds = exp2f(s * sl2 - lse2) * (dp - Drow);
+        int seq = 0;
+        bool ok = true;
+        for (int x = 0; x < n_items && ok; ++x) {
+            for (int kv = 0; kv < 2; ++kv, ++seq) {
+                const int st = seq % kDqStages;
+                if (!wait_all(&bars->empty[st], ((seq / kDqStages) & 1) ^ 1)) {
+                    if (lead) flag_timeout(p.status, bars);
+                    ok = false;
+                    break;
+                }
+                ptx::mbar_arrive_expect_tx_lead(&bars->full[st], kTile, lead);
+                uint8_t* dst = sRing + st * kTile;
+                for (int hf = 0; hf < 2; ++hf) {
+                    if (x < n_kv)
+                        ptx::tma_load_4d_lead(dst + hf * kHalf, kv ? &p.tm_v : &p.tm_k, &bars->full[st], hf * 64,
+                                              kvh, x * kBK, b, lead);
+                    else
+                        ptx::tma_load_4d_lead(dst + hf * kHalf, kv ? &p.tm_vd : &p.tm_kd, &bars->full[st], hf * 64,
+                                              kvh, t0 * p.Ld + (x - n_kv) * kBK, b, lead);
+                }
+            }
+        }
+        ptx::mbar_wait(&bars->kv_full, 0, 0, nullptr);
+        for (int s = (seq > kDqStages ? seq - kDqStages : 0); s < seq; ++s)
+            ptx::mbar_wait(&bars->full[s % kDqStages], (s / kDqStages) & 1, 0, nullptr);
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        const uint32_t lead = lane == 0;
+        constexpr uint32_t idesc_ss = ptx::idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint32_t idesc_ts = ptx::idesc_bf16_f32(128, kD, 0, 1);
+        const uint64_t dQk = kdesc(ptx::smem_u32(sQ)), dOk = kdesc(ptx::smem_u32(sDO));
+        const uint32_t aRing = ptx::smem_u32(sRing);
+        bool ok = wait_all(&bars->kv_full, 0);
+        if (!ok && lead) flag_timeout(p.status, bars);
+        ptx::tc_fence_after();
+        // ring slots: item x has K at 2x, V at 2x+1
+        auto issue_s = [&](int x) {  // S(x) = Q K(x)^T into R[x % 2]
+            const int sk = 2 * x;
+            if (!wait_all(&bars->full[sk % kDqStages], (sk / kDqStages) & 1)) return false;
+            ptx::tc_fence_after();
+            const uint64_t kk = kdesc(aRing + (sk % kDqStages) * kTile);
 #pragma unroll
-        for (int e = 0; e < NP; ++e) {
-            acc[e].x = fmaf(ds, kr[e].x, acc[e].x);
-            acc[e].y = fmaf(ds, kr[e].y, acc[e].y);
+            for (int k = 0; k < kD / 16; ++k)
+                ptx::mma_ss_lead(tmem + (x & 1) * 128, dQk + koff(k), kk + koff(k), idesc_ss, k > 0, lead);
+            ptx::mma_commit_lead(&bars->s_full, lead);
+            return true;
+        };
+        auto issue_dp = [&](int x) {  // dP(x) = dO V(x)^T into R[(x + 1) % 2]
+            const int sv = 2 * x + 1;
+            if (!wait_all(&bars->full[sv % kDqStages], (sv / kDqStages) & 1)) return false;
+            ptx::tc_fence_after();
+            const uint64_t vk = kdesc(aRing + (sv % kDqStages) * kTile);
+#pragma unroll
+            for (int k = 0; k < kD / 16; ++k)
+                ptx::mma_ss_lead(tmem + ((x + 1) & 1) * 128, dOk + koff(k), vk + koff(k), idesc_ss, k > 0, lead);
+            ptx::mma_commit_lead(&bars->dp_full, lead);
+            return true;
+        };
+        if (ok) ok = issue_s(0) && issue_dp(0);
+        for (int x = 0; x < n_items && ok; ++x) {
+            // dS(x) is in R[x % 2]; the compute warps have read dP(x) from
+            // R[(x + 1) % 2], which S(x + 1) may now overwrite.
+            if (!wait_all(&bars->p_full, x & 1)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            if (x + 1 < n_items && !issue_s(x + 1)) {
+                ok = false;
+                break;
+            }
+            const int sk = 2 * x;
+            const uint64_t km = mndesc(aRing + (sk % kDqStages) * kTile);
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k)
+                ptx::mma_ts_lead(tmem + 256, tmem + (x & 1) * 128 + k * 8, km + mnoff(k), idesc_ts,
+                                 (x > 0 || k > 0) ? 1u : 0u, lead);
+            // K(x), V(x) are no longer needed
+            ptx::mma_commit_lead(&bars->empty[sk % kDqStages], lead);
+            ptx::mma_commit_lead(&bars->empty[(sk + 1) % kDqStages], lead);
+            // dP(x + 1) into R[x % 2], after dQ has read dS(x) there
+            if (x + 1 < n_items && !issue_dp(x + 1)) {
+                ok = false;
+                break;
+            }
+        }
+        if (!ok && lead) flag_timeout(p.status, bars);
+        if (ok) ptx::mma_commit_lead(&bars->fin, lead);
+        ptx::mma_commit_lead(&bars->drain, lead);
+        ptx::mbar_wait(&bars->drain, 0, 0, nullptr);
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ compute warps
+        const int r = warp * 32 + lane;  // TMEM lane = query row (token-major)
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const int tt = r / p.G;          // token within the tile
+        const int t = t0 + tt, h = kvh * p.G + r % p.G;
+        const bool row_ok = t < p.T;
+        float lse2 = INFINITY, Drow = 0.f;
+        if (row_ok) {
+            const long long ix = ((long long)b * p.Hq + h) * p.T + t;
+            lse2 = p.lse[ix] * kLog2e;
+            Drow = p.rowD[ix];
+        }
+        const float sl2 = p.sl2;
+        bool ok = true;
+        for (int x = 0; x < n_items; ++x) {
+            const uint32_t rS = tmem + lane_off + (x & 1) * 128;        // S(x), then dS(x)
+            const uint32_t rP = tmem + lane_off + ((x + 1) & 1) * 128;  // dP(x)
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s_full, x & 1, p.wait_limit, abort_flag))) {
+                flag_timeout(p.status, bars);
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            float pr[128];
+            {
+                uint32_t su[128];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) ptx::tmem_ld32(rS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&su[c * 32]));
+                ptx::tmem_wait_ld();
+                int lo, hi;  // visible columns of this row
+                if (x < n_kv) {
+                    lo = 0;
+                    hi = t - x * kBK + 1;  // keys <= t
+                } else {
+                    lo = tt * p.Ld - (x - n_kv) * kBK;  // the row's own depth rows
+                    hi = lo + p.Ld;
+                }
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    const float e = ptx::ex2(fmaf(__uint_as_float(su[c]), sl2, -lse2));
+                    pr[c] = (c >= lo && c < hi) ? e : 0.f;
+                }
+            }
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->dp_full, x & 1, p.wait_limit, abort_flag))) {
+                flag_timeout(p.status, bars);
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t dr[32];
+                ptx::tmem_ld32(rP + 32 * c, dr);
+                ptx::tmem_wait_ld();
+                uint32_t dd[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float d0 = pr[32 * c + 2 * e] * (__uint_as_float(dr[2 * e]) - Drow);
+                    const float d1 = pr[32 * c + 2 * e + 1] * (__uint_as_float(dr[2 * e + 1]) - Drow);
+                    dd[e] = ptx::pack_bf16x2(d0, d1);
+                }
+                ptx::tmem_st16(rS + 16 * c, dd);  // over S(x), already read
+            }
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&bars->p_full);
+        }
+        if (ok && !__all_sync(0xffffffffu, ptx::mbar_wait(&bars->fin, 0, p.wait_limit, abort_flag))) {
+            flag_timeout(p.status, bars);
+            ok = false;
+        }
+        ptx::tc_fence_after();
+        if (ok) {
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.dq) + (((long long)b * p.T + (row_ok ? t : 0)) * p.Hq + h) * kD;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                ptx::tmem_ld32(tmem + lane_off + 256 + 32 * c, o);
+                ptx::tmem_wait_ld();
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    w[e] = ptx::pack_bf16x2(__uint_as_float(o[2 * e]) * p.scale, __uint_as_float(o[2 * e + 1]) * p.scale);
+                if (row_ok) {
+                    uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                }
+            }
         }
     }
-    if (valid) {
-        float* dst = a.dq_acc + rc * kD;
-#pragma unroll
-        for (int e = 0; e < NP; ++e) {
-            const int c = 2 * (TPR * e + u);
-            *reinterpret_cast<float2*>(dst + c) = make_float2(acc[e].x * f.scale, acc[e].y * f.scale);
-        }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 512);
     }
 }
 
-// fp32 accumulator -> bf16 (dq, dk, dv).
-__global__ void dq_convert_kernel(const float4* acc, uint2* dq, long long n4) {
+// fp32 accumulator -> bf16 (dk, dv).
+__global__ void acc_to_bf16_kernel(const float4* acc, uint2* out, long long n4) {
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
          i += (long long)gridDim.x * blockDim.x) {
         const float4 v = acc[i];
-        dq[i] = make_uint2(ptx::pack_bf16x2(v.x, v.y), ptx::pack_bf16x2(v.z, v.w));
+        out[i] = make_uint2(ptx::pack_bf16x2(v.x, v.y), ptx::pack_bf16x2(v.z, v.w));
     }
 }
 
@@ -491,7 +646,8 @@ bool bwd_tc_supported(const BwdArgs& a) {
     const FwdArgs& f = a.f;
     if (f.dtype != MODA_BF16 || f.d != kD) return false;
     if (f.G < 1 || f.G > 128 || 128 % f.G) return false;
-    if (!a.dq_acc) return false;
+    if (!a.dk_acc || !a.dv_acc) return false;
+    if ((long long)f.T * f.Ld >= (1LL << 31)) return false;
     const Strides4 sq = strides_q(f.T, f.Hq, f.d), skv = strides_q(f.T, f.Hkv, f.d);
     const Strides5 sdep = strides_depth_native(f.T, f.Ld, f.Hkv, f.d);
     if (f.sq.sb != sq.sb || f.sq.st != sq.st || f.sq.sh != sq.sh) return false;
@@ -506,74 +662,94 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s) {
     const FwdArgs& f = a.f;
     cudaError_t e = launch_bwd_rowdot(a, s);
     if (e != cudaSuccess) return e;
-    {
-        const long long rows = (long long)f.B * f.T * f.Hq;
-        bwd_depth_dq_kernel<<<(unsigned)((rows + 63) / 64), 256, 0, s>>>(a);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
     if ((e = launch_bwd_depth_dkv(a, s)) != cudaSuccess) return e;
 
-    TcBwdParams p;
-    memset(&p, 0, sizeof(p));
     const int G = f.G, n = 128 / G;
+    int gshift = 0;
+    while ((1 << gshift) < G) ++gshift;
     const cuuint64_t es = 2;
+    CUtensorMap tm_q, tm_do, tm_k, tm_v, tm_kd, tm_vd;
     {
         const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)f.Hq, (cuuint64_t)f.T, (cuuint64_t)f.B};
         const cuuint64_t st[3] = {kD * es, (cuuint64_t)f.Hq * kD * es, (cuuint64_t)f.T * f.Hq * kD * es};
         const cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)n, 1};
-        if (!make_tmap_bf16_4d(&p.tm_q, f.q, dims, st, box)) return cudaErrorInvalidValue;
-        if (!make_tmap_bf16_4d(&p.tm_do, a.dout, dims, st, box)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16_4d(&tm_q, f.q, dims, st, box)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16_4d(&tm_do, a.dout, dims, st, box)) return cudaErrorInvalidValue;
     }
     {
         const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)f.Hkv, (cuuint64_t)f.T, (cuuint64_t)f.B};
         const cuuint64_t st[3] = {kD * es, (cuuint64_t)f.Hkv * kD * es, (cuuint64_t)f.T * f.Hkv * kD * es};
         const cuuint32_t box[4] = {64, 1, (cuuint32_t)kBK, 1};
-        if (!make_tmap_bf16_4d(&p.tm_k, f.k, dims, st, box)) return cudaErrorInvalidValue;
-        if (!make_tmap_bf16_4d(&p.tm_v, f.v, dims, st, box)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16_4d(&tm_k, f.k, dims, st, box)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16_4d(&tm_v, f.v, dims, st, box)) return cudaErrorInvalidValue;
     }
-    p.lse = f.lse;
-    p.rowD = a.rowD;
-    p.dq_acc = a.dq_acc;
-    p.dk_acc = a.dk_acc;
-    p.dv_acc = a.dv_acc;
-    p.B = f.B; p.T = f.T; p.Hq = f.Hq; p.Hkv = f.Hkv; p.G = G; p.n = n;
-    p.nkt = (f.T + kBK - 1) / kBK;
-    // Query tiles per CTA: enough CTAs for ~4 waves over the SMs, at least
-    // 16 tiles each so the dK / dV flush stays small against the work.
+    if (f.Ld > 0) {
+        const cuuint64_t rows = (cuuint64_t)f.T * f.Ld;
+        const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)f.Hkv, rows, (cuuint64_t)f.B};
+        const cuuint64_t st[3] = {kD * es, (cuuint64_t)f.Hkv * kD * es, rows * f.Hkv * kD * es};
+        const cuuint32_t box[4] = {64, 1, (cuuint32_t)kBK, 1};
+        if (!make_tmap_bf16_4d(&tm_kd, f.kd, dims, st, box)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16_4d(&tm_vd, f.vd, dims, st, box)) return cudaErrorInvalidValue;
+    } else {
+        tm_kd = tm_k;
+        tm_vd = tm_v;
+    }
+    const int sms = sm_count();
+
+    // ---- dk, dv
+    DkvParams pk;
+    memset(&pk, 0, sizeof(pk));
+    pk.tm_q = tm_q; pk.tm_do = tm_do; pk.tm_k = tm_k; pk.tm_v = tm_v;
+    pk.lse = f.lse; pk.rowD = a.rowD; pk.dk_acc = a.dk_acc; pk.dv_acc = a.dv_acc;
+    pk.B = f.B; pk.T = f.T; pk.Hq = f.Hq; pk.Hkv = f.Hkv; pk.G = G; pk.n = n; pk.gshift = gshift;
+    pk.sl2 = f.scale * kLog2e; pk.scale = f.scale;
+    pk.status = f.status; pk.wait_limit = f.wait_limit;
+    const int nkt = (f.T + kBK - 1) / kBK;
     {
+        // query tiles per CTA: ~4 waves over the SMs, at least 16 tiles each
         long long steps = 0;
-        for (int kt = 0; kt < p.nkt; ++kt) steps += (f.T - kt * kBK + n - 1) / n;
+        for (int kt = 0; kt < nkt; ++kt) steps += (f.T - kt * kBK + n - 1) / n;
         steps *= (long long)f.B * f.Hkv;
-        long long qc = (steps + 4LL * sm_count() - 1) / (4LL * sm_count());
-        if (qc < 16) qc = 16;
-        p.qchunk = (int)qc;
+        long long qc = (steps + 4LL * sms - 1) / (4LL * sms);
+        pk.qchunk = (int)(qc < 16 ? 16 : qc);
     }
-    p.sl2 = f.scale * kLog2e;
-    p.scale = f.scale;
-    p.status = f.status;
-    p.wait_limit = f.wait_limit;
-    if ((e = cudaFuncSetAttribute(moda_bwd_seq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  kSmemBytes)) != cudaSuccess)
-        return e;
     const size_t kv_bytes = (size_t)f.B * f.T * f.Hkv * kD * sizeof(float);
     if ((e = cudaMemsetAsync(a.dk_acc, 0, kv_bytes, s)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(a.dv_acc, 0, kv_bytes, s)) != cudaSuccess) return e;
-    const int n_chunks = ((f.T + n - 1) / n + p.qchunk - 1) / p.qchunk;
-    dim3 grid(p.nkt, n_chunks, f.B * f.Hkv);
-    moda_bwd_seq_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(p);
+    if ((e = cudaFuncSetAttribute(moda_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDkvSmem)) !=
+        cudaSuccess)
+        return e;
+    const int n_chunks = ((f.T + n - 1) / n + pk.qchunk - 1) / pk.qchunk;
+    moda_bwd_dkdv_kernel<<<dim3(nkt, n_chunks, f.B * f.Hkv), kThreads, kDkvSmem, s>>>(pk);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-    auto convert = [&](const float* acc, void* dst, long long elems) {
-        const long long n4 = elems / 4;
-        long long blocks = (n4 + 255) / 256;
-        if (blocks > (long long)sm_count() * 8) blocks = (long long)sm_count() * 8;
-        dq_convert_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(acc),
-                                                           static_cast<uint2*>(dst), n4);
-        return cudaGetLastError();
-    };
-    if ((e = convert(a.dq_acc, a.dq, (long long)f.B * f.T * f.Hq * kD)) != cudaSuccess) return e;
-    if ((e = convert(a.dk_acc, a.dk, (long long)f.B * f.T * f.Hkv * kD)) != cudaSuccess) return e;
-    return convert(a.dv_acc, a.dv, (long long)f.B * f.T * f.Hkv * kD);
+    // ---- dq
+    DqParams pq;
+    memset(&pq, 0, sizeof(pq));
+    pq.tm_q = tm_q; pq.tm_do = tm_do; pq.tm_k = tm_k; pq.tm_v = tm_v; pq.tm_kd = tm_kd; pq.tm_vd = tm_vd;
+    pq.lse = f.lse; pq.rowD = a.rowD; pq.dq = a.dq;
+    pq.B = f.B; pq.T = f.T; pq.Hq = f.Hq; pq.Hkv = f.Hkv; pq.G = G; pq.n = n; pq.Ld = f.Ld;
+    pq.nqt = (f.T + n - 1) / n;
+    pq.sl2 = f.scale * kLog2e; pq.scale = f.scale;
+    pq.status = f.status; pq.wait_limit = f.wait_limit;
+    if ((e = cudaFuncSetAttribute(moda_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem)) !=
+        cudaSuccess)
+        return e;
+    const long long grid_q = (long long)pq.nqt * f.B * f.Hkv;
+    if (grid_q > 0x7fffffffLL) return cudaErrorInvalidValue;
+    moda_bwd_dq_kernel<<<(unsigned)grid_q, kThreads, kDqSmem, s>>>(pq);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    // ---- dk, dv to bf16
+    const long long n4 = (long long)f.B * f.T * f.Hkv * kD / 4;
+    long long blocks = (n4 + 255) / 256;
+    if (blocks > (long long)sms * 8) blocks = (long long)sms * 8;
+    acc_to_bf16_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(a.dk_acc),
+                                                        static_cast<uint2*>(a.dk), n4);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    acc_to_bf16_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(a.dv_acc),
+                                                        static_cast<uint2*>(a.dv), n4);
+    return cudaGetLastError();
 }
 
 }  // namespace moda

@@ -46,7 +46,6 @@ struct BwdArgs {
     void* dkd;
     void* dvd;
     float* rowD;            // [B, Hq, T] fp32 workspace: <dout, out>
-    float* dq_acc;          // [B, T, Hq, d] fp32 workspace (tensor-core path only)
     float* dk_acc;          // [B, T, Hkv, d] fp32 workspace (tensor-core path only)
     float* dv_acc;          // [B, T, Hkv, d] fp32 workspace (tensor-core path only)
 };

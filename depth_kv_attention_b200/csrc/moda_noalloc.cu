@@ -95,7 +95,6 @@ extern "C" moda_status moda_bwd_noalloc(const void* q, const void* k, const void
     // The backward's first kernel writes every D it later reads, so the
     // previous call's contents need no clearing.
     a.rowD = static_cast<float*>(scratch);
-    a.dq_acc = nullptr;
     cudaError_t e = launch_bwd_simt(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
 }

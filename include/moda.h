@@ -114,8 +114,7 @@ moda_status moda_fwd_ex(const void* q, const void* k, const void* v,
 /*
  * moda_bwd_workspace_bytes — bytes of fp32 scratch moda_bwd needs for this
  * shape: row statistics D [B,Hq,T] and, for bf16 (tensor-core path), fp32
- * accumulators of dq [B,T,Hq,d], dk and dv [B,T,Hkv,d]. Returns 0 for an
- * invalid shape.
+ * accumulators of dk and dv [B,T,Hkv,d]. Returns 0 for an invalid shape.
  */
 size_t moda_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int Ld,
                                 moda_dtype dtype);

@@ -79,8 +79,8 @@ def test_bwd_validation():
 
 
 def test_workspace_and_pack_sizes():
-    # fp32 row statistics [B,Hq,T] (256-byte rounded) + fp32 dq, dk, dv accumulators for bf16
-    assert moda._c_bwd_ws(1, 8, 4, 2, 64, 2, 0) == 256 + 8 * (4 + 2 * 2) * 64 * 4
+    # fp32 row statistics [B,Hq,T] (256-byte rounded) + fp32 dk, dv accumulators for bf16
+    assert moda._c_bwd_ws(1, 8, 4, 2, 64, 2, 0) == 256 + 8 * (2 * 2) * 64 * 4
     assert moda._c_bwd_ws(1, 8, 4, 2, 64, 2, 1) == 256
     assert moda._c_bwd_ws(1, 8, 3, 2, 64, 2, 0) == 0
     assert moda._c_pack_bytes(2, 5, 3, 128, 7, 0) == 2 * 2 * 5 * 7 * 3 * 128 * 2
