@@ -10,9 +10,10 @@
 //
 // Launch sequence (one stream):
 //   1. D = rowsum(dout * out)                      (SIMT, shared with the SIMT path)
-//   2. dkd, dvd                                     (SIMT, shared with the SIMT path)
-//   3. dk, dv: KV-major tensor-core kernel; partial sums of a key tile over a
+//   2. dk, dv: KV-major tensor-core kernel; partial sums of a key tile over a
 //      chunk of query tiles go to fp32 accumulators with vector reductions
+//   3. dkd, dvd: the same kernel with 128-row depth chunks as the key tiles
+//      and a same-token mask (each depth row owned by one CTA, bf16 stores)
 //   4. dq: query-major tensor-core kernel over the causal key tiles and the
 //      query tile's own depth chunks; dq accumulates in TMEM and is written
 //      once, in bf16 (no dq reductions between CTAs)
@@ -109,11 +110,14 @@ __device__ __forceinline__ void init_bars(Bars* bars, int stages) {
 
 // ===================================================================== dk, dv
 struct DkvParams {
-    CUtensorMap tm_q, tm_do, tm_k, tm_v;
+    CUtensorMap tm_q, tm_do, tm_k, tm_v;  // in depth mode tm_k / tm_v map kd / vd
     const float* lse;
     const float* rowD;
-    float* dk_acc;  // [B,T,Hkv,d] fp32, zeroed before the launch
+    float* dk_acc;  // sequence mode: [B,T,Hkv,d] fp32, zeroed before the launch
     float* dv_acc;
+    void* dkd;      // depth mode: [B,T,Ld,Hkv,d] bf16 outputs
+    void* dvd;
+    int depth_mode, Ld;
     int B, T, Hq, Hkv, G, n, gshift, qchunk;
     float sl2, scale;
     unsigned int* status;
@@ -124,8 +128,15 @@ constexpr int kDkvSmem = 2 * kTile + kDkvStages * 2 * kTile + 2 * 128 * 4 + 256 
 static_assert(kDkvSmem <= 232448, "shared memory per CTA");
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
-// One CTA per (key tile = blockIdx.x, chunk of query tokens = blockIdx.y,
-// (b, kv-head) = blockIdx.z). TMEM: S^T | dP^T | dV | dK, 128 columns each.
+// Sequence mode: one CTA per (key tile = blockIdx.x, chunk of query tokens =
+// blockIdx.y, (b, kv-head) = blockIdx.z), causal mask, partial sums reduced
+// into fp32 accumulators.
+// Depth mode (the depth keys' gradients dkd, dvd): the "key tile" is the
+// 128-row depth chunk blockIdx.x of the [B, T*Ld, Hkv, d] view, the query
+// tiles are those holding the chunk's tokens, the mask keeps each depth row
+// to its own token's G heads, and since one CTA owns every row of its chunk
+// the results are written directly in bf16.
+// TMEM: S^T | dP^T | dV | dK, 128 columns each.
 // Per query tile: S^T = K Q^T, dP^T = V dO^T; the compute warps (thread =
 // key) form P^T and dS^T in bf16 over S^T / dP^T; dV += P^T dO and
 // dK += dS^T Q take them as TMEM A operands. The next tile's S^T / dP^T
@@ -143,16 +154,24 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     volatile int* abort_flag = &bars->abort_flag;
     const int b = blockIdx.z / p.Hkv, kvh = blockIdx.z % p.Hkv;
-    const int j0 = blockIdx.x * kBK;
+    const int j0 = blockIdx.x * kBK;  // first key row (sequence) or depth row (depth mode)
     const int n = p.n;
-    // A chunk is qchunk query tiles of absolute tokens [c*qchunk*n, ...); the
-    // CTAs in flight at once cover one or two chunks. Key tiles that no row of
-    // the chunk can see exit at once.
-    const int c_lo = blockIdx.y * p.qchunk * n;
-    const int c_hi = min(p.T, (blockIdx.y + 1) * p.qchunk * n);
-    const int t_first = max(j0, c_lo);  // a multiple of n
-    if (t_first >= c_hi) return;
-    const int nq = (c_hi - t_first + n - 1) / n;
+    int t_first, nq;
+    if (p.depth_mode) {
+        // tokens whose depth rows meet [j0, j0 + 128), whole query tiles
+        const int last_row = min(j0 + kBK, p.T * p.Ld) - 1;
+        t_first = (j0 / p.Ld) / n * n;
+        nq = (last_row / p.Ld - t_first) / n + 1;
+    } else {
+        // A chunk is qchunk query tiles of absolute tokens [c*qchunk*n, ...);
+        // the CTAs in flight at once cover one or two chunks. Key tiles that
+        // no row of the chunk can see exit at once.
+        const int c_lo = blockIdx.y * p.qchunk * n;
+        const int c_hi = min(p.T, (blockIdx.y + 1) * p.qchunk * n);
+        t_first = max(j0, c_lo);  // a multiple of n
+        if (t_first >= c_hi) return;
+        nq = (c_hi - t_first + n - 1) / n;
+    }
 
     if (threadIdx.x == 0) init_bars(bars, kDkvStages);
     if (warp == 0) {
@@ -281,9 +300,18 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
                 break;
             }
             ptx::tc_fence_after();
-            // key j is visible to row rr iff j <= tq0 + (rr >> gshift): rows
-            // rr < (j - tq0) << gshift are masked.
-            const int mask_below = j > tq0 ? (j - tq0) << gshift : 0;
+            // Visible rows rr form a range [lo_r, hi_r): sequence mode, key j
+            // is seen by rows of tokens tq0 + (rr >> gshift) >= j; depth mode,
+            // depth row j is seen only by the rows of its own token j / Ld.
+            int lo_r, hi_r;
+            if (p.depth_mode) {
+                const int td = j < p.T * p.Ld ? j / p.Ld : -1;
+                lo_r = (td - tq0) * p.G;
+                hi_r = td < 0 ? lo_r : lo_r + p.G;
+            } else {
+                lo_r = j > tq0 ? (j - tq0) << gshift : 0;
+                hi_r = 128;
+            }
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t sr[32], dr[32];
@@ -298,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
                     for (int u = 0; u < 2; ++u) {
                         const int rr = 32 * c + 2 * e2 + u;
                         float pr = ptx::ex2(fmaf(__uint_as_float(sr[2 * e2 + u]), sl2, -st_lse[rr]));
-                        if (rr < mask_below) pr = 0.f;
+                        if (rr < lo_r || rr >= hi_r) pr = 0.f;
                         pv[u] = pr;
                         dv[u] = pr * (__uint_as_float(dr[2 * e2 + u]) - st_D[rr]);
                     }
@@ -322,7 +350,35 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
             }
         }
         ptx::tc_fence_after();
-        if (ok) {
+        if (ok && p.depth_mode) {
+            // dkd (scaled) and dvd of this chunk's depth rows, written directly
+            const bool valid = j < p.T * p.Ld;
+            const long long off = (((long long)b * p.T * p.Ld + (valid ? j : 0)) * p.Hkv + kvh) * kD;
+            __nv_bfloat16* dvr = static_cast<__nv_bfloat16*>(p.dvd) + off;
+            __nv_bfloat16* dkr = static_cast<__nv_bfloat16*>(p.dkd) + off;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t a[32], g[32];
+                ptx::tmem_ld32(tmem + lane_off + 256 + 32 * c, a);
+                ptx::tmem_ld32(tmem + lane_off + 384 + 32 * c, g);
+                ptx::tmem_wait_ld();
+                uint32_t wa[16], wg[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    wa[e] = ptx::pack_bf16x2(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]));
+                    wg[e] = ptx::pack_bf16x2(__uint_as_float(g[2 * e]) * p.scale, __uint_as_float(g[2 * e + 1]) * p.scale);
+                }
+                if (valid) {
+                    uint4* da = reinterpret_cast<uint4*>(dvr + 32 * c);
+                    uint4* dg = reinterpret_cast<uint4*>(dkr + 32 * c);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        da[v] = make_uint4(wa[4 * v], wa[4 * v + 1], wa[4 * v + 2], wa[4 * v + 3]);
+                        dg[v] = make_uint4(wg[4 * v], wg[4 * v + 1], wg[4 * v + 2], wg[4 * v + 3]);
+                    }
+                }
+            }
+        } else if (ok) {
             // This chunk's partial dK (scaled) and dV, added into the fp32
             // accumulators (other chunks of the same key tile add theirs).
             const bool valid = j < p.T;
@@ -662,8 +718,6 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s) {
     const FwdArgs& f = a.f;
     cudaError_t e = launch_bwd_rowdot(a, s);
     if (e != cudaSuccess) return e;
-    if ((e = launch_bwd_depth_dkv(a, s)) != cudaSuccess) return e;
-
     const int G = f.G, n = 128 / G;
     int gshift = 0;
     while ((1 << gshift) < G) ++gshift;
@@ -722,6 +776,21 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s) {
     const int n_chunks = ((f.T + n - 1) / n + pk.qchunk - 1) / pk.qchunk;
     moda_bwd_dkdv_kernel<<<dim3(nkt, n_chunks, f.B * f.Hkv), kThreads, kDkvSmem, s>>>(pk);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    // ---- dkd, dvd: the same kernel over the depth chunks
+    if (f.Ld > 0) {
+        DkvParams pd = pk;
+        pd.tm_k = tm_kd;
+        pd.tm_v = tm_vd;
+        pd.depth_mode = 1;
+        pd.Ld = f.Ld;
+        pd.dkd = a.dkd;
+        pd.dvd = a.dvd;
+        const long long chunks = ((long long)f.T * f.Ld + kBK - 1) / kBK;
+        if (chunks > 0x7fffffffLL) return cudaErrorInvalidValue;
+        moda_bwd_dkdv_kernel<<<dim3((unsigned)chunks, 1, f.B * f.Hkv), kThreads, kDkvSmem, s>>>(pd);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
 
     // ---- dq
     DqParams pq;
