@@ -46,6 +46,17 @@ constexpr int kThreads = 192;     // warps 0-3 compute, 4 TMA producer, 5 MMA
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr float kLog2e = 1.4426950408889634f;
+// Of every 8 column pairs, pairs kBwdPolyFrom..7 take exp2 from the FMA-pipe
+// polynomial, the rest from MUFU (in these kernels the exponentials sit on
+// the critical path of one compute warp per SM sub-partition).
+#ifndef MODA_BWD_POLY_FROM
+#define MODA_BWD_POLY_FROM 8
+#endif
+constexpr int kBwdPolyFrom = MODA_BWD_POLY_FROM;
+__device__ __forceinline__ float2 exp2_pair(float2 x, int pair) {
+    if ((pair & 7) >= kBwdPolyFrom) return ptx::exp2_poly2(x);
+    return make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
+}
 
 __device__ __forceinline__ uint64_t kdesc(uint32_t tile) { return ptx::umma_desc_sw128(tile, 16, 1024); }
 __device__ __forceinline__ uint64_t mndesc(uint32_t tile) { return ptx::umma_desc_sw128(tile, kHalf, 1024); }
@@ -322,10 +333,14 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
 #pragma unroll
                 for (int e2 = 0; e2 < 16; ++e2) {
                     float pv[2], dv[2];
+                    const int r0 = 32 * c + 2 * e2;
+                    const float2 ex = exp2_pair(make_float2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -st_lse[r0]),
+                                                            fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -st_lse[r0 + 1])),
+                                                e2);
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const int rr = 32 * c + 2 * e2 + u;
-                        float pr = ptx::ex2(fmaf(__uint_as_float(sr[2 * e2 + u]), sl2, -st_lse[rr]));
+                        const int rr = r0 + u;
+                        float pr = u ? ex.y : ex.x;
                         if (rr < lo_r || rr >= hi_r) pr = 0.f;
                         pv[u] = pr;
                         dv[u] = pr * (__uint_as_float(dr[2 * e2 + u]) - st_D[rr]);
@@ -618,9 +633,12 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
                     hi = lo + p.Ld;
                 }
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    const float e = ptx::ex2(fmaf(__uint_as_float(su[c]), sl2, -lse2));
-                    pr[c] = (c >= lo && c < hi) ? e : 0.f;
+                for (int c = 0; c < 128; c += 2) {
+                    const float2 e = exp2_pair(make_float2(fmaf(__uint_as_float(su[c]), sl2, -lse2),
+                                                           fmaf(__uint_as_float(su[c + 1]), sl2, -lse2)),
+                                               c / 2);
+                    pr[c] = (c >= lo && c < hi) ? e.x : 0.f;
+                    pr[c + 1] = (c + 1 >= lo && c + 1 < hi) ? e.y : 0.f;
                 }
             }
             if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->dp_full, x & 1, p.wait_limit, abort_flag))) {
