@@ -25,7 +25,8 @@ from dataclasses import dataclass, replace
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "sample_rows", "workload"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "sample_rows", "workload", "make_depth_sel",
+           "pack_depth_sel"]
 
 
 @dataclass(frozen=True)
@@ -130,3 +131,37 @@ def sample_rows(w: Workload, n_rows: int = 256, n_head: int = 16) -> list[int]:
     pool = torch.arange(n_head, T - 1)
     pick = pool[torch.randperm(pool.numel(), generator=g)[:rest_n]].tolist()
     return sorted(set(head + pick + [T - 1]))
+
+
+def make_depth_sel(w: Workload, kind: str = "random", density: float = 0.5, seed_offset: int = 2):
+    """Seeded per-token depth selection [B, T, Ld] (bool).
+
+    kind "random": each depth entry kept with probability ``density``;
+    "window": each token keeps a contiguous window of its most recent
+    entries (the last W of Ld, W uniform in [0, Ld]); "all"; "none".
+    """
+    g = torch.Generator("cpu")
+    g.manual_seed(w.seed + seed_offset)
+    shape = (w.B, w.T, w.Ld)
+    if kind == "all":
+        return torch.ones(shape, dtype=torch.bool)
+    if kind == "none":
+        return torch.zeros(shape, dtype=torch.bool)
+    if kind == "random":
+        return torch.rand(shape, generator=g) < density
+    if kind == "window":
+        width = torch.randint(0, w.Ld + 1, (w.B, w.T, 1), generator=g)
+        i = torch.arange(w.Ld).view(1, 1, -1)
+        return i >= (w.Ld - width)
+    raise ValueError(kind)
+
+
+def pack_depth_sel(sel) -> torch.Tensor:
+    """[B, T, Ld] bool -> [B, T] int64 bit masks (bit i = entry i), Ld <= 64."""
+    B, T, Ld = sel.shape
+    if Ld > 64:
+        raise ValueError("bit masks hold at most 64 depth entries")
+    bits = torch.zeros((B, T), dtype=torch.int64)
+    for i in range(Ld):
+        bits |= sel[:, :, i].to(torch.int64) << i
+    return bits

@@ -31,6 +31,12 @@ Sources:
   * "Mixture-of-Depths Attention" (gist.science, French technical summary),
     §2 "Méthodologie", Opération: one unified softmax over sequence and depth.
 
+Selected depth (the pages' future-work item, "Mixture-of-Depths Attention",
+gist.science German summary §5: bounded depth-KV slots, e.g. a sliding window
+over layers or a dynamic selection): an optional ``depth_sel`` [B, T, Ld] of
+booleans keeps depth entry i of token t only where depth_sel[b,t,i] is true;
+the other depth logits leave the softmax (as if that slot were absent).
+
 Readings where the pages are silent (each also listed in the design doc):
   * the depth logits take the same ``scale`` as the sequence logits (the §1.2
     formula divides the whole concatenation by sqrt(d));
@@ -70,19 +76,27 @@ def _dims(q, k, kd):
     return B, T, Hq, Hkv, Hq // Hkv, d, Ld
 
 
-def _concat_logits(qr, kseq, kdep, scale, ts):
+def _concat_logits(qr, kseq, kdep, scale, ts, sel=None):
     """Concatenated logit rows [sequence || depth] for query rows ``qr``.
 
     qr   [R, d]   query vectors of positions ``ts`` (one head)
     kseq [J, d]   sequence keys 0..J-1 of the head's kv-head
     kdep [R, Ld, d] depth keys of the SAME positions ``ts``
-    Returns s [R, J + Ld] with -inf where the causal mask hides a key.
+    sel  [R, Ld] booleans or None: depth entries kept for each row's position
+    Returns s [R, J + Ld] with -inf where the causal mask hides a key or a
+    depth entry is not selected.
     """
     s_seq = scale * (qr @ kseq.T)                            # [R, J]
     j = np.arange(kseq.shape[0])
     s_seq = np.where(j[None, :] <= np.asarray(ts)[:, None], s_seq, -np.inf)
     s_dep = scale * np.einsum("rc,ric->ri", qr, kdep)        # [R, Ld]
+    if sel is not None:
+        s_dep = np.where(sel, s_dep, -np.inf)
     return np.concatenate([s_seq, s_dep], axis=1)
+
+
+def _sel(depth_sel, b, t0, t1):
+    return None if depth_sel is None else np.asarray(depth_sel[b, t0:t1], dtype=bool)
 
 
 def _softmax_rows(s):
@@ -93,8 +107,10 @@ def _softmax_rows(s):
     return e / z, (m + np.log(z))[:, 0]
 
 
-def forward(q, k, v, kd, vd, scale: float, row_block: int = 256):
-    """Full MoDA forward. Returns (out [B,T,Hq,d], lse [B,Hq,T]) in float64."""
+def forward(q, k, v, kd, vd, scale: float, row_block: int = 256, depth_sel=None):
+    """Full MoDA forward. Returns (out [B,T,Hq,d], lse [B,Hq,T]) in float64.
+
+    ``depth_sel`` (optional, [B,T,Ld] bool): depth entries each position keeps."""
     q, k, v, kd, vd = (to_f64(x) for x in (q, k, v, kd, vd))
     B, T, Hq, Hkv, G, d, Ld = _dims(q, k, kd)
     out = np.empty((B, T, Hq, d))
@@ -106,7 +122,7 @@ def forward(q, k, v, kd, vd, scale: float, row_block: int = 256):
                 t1 = min(T, t0 + row_block)
                 ts = np.arange(t0, t1)
                 s = _concat_logits(q[b, t0:t1, h], k[b, :t1, g],
-                                   kd[b, t0:t1, :, g], scale, ts)
+                                   kd[b, t0:t1, :, g], scale, ts, _sel(depth_sel, b, t0, t1))
                 p, l = _softmax_rows(s)
                 vals = p[:, :t1] @ v[b, :t1, g]
                 vals += np.einsum("ri,ric->rc", p[:, t1:], vd[b, t0:t1, :, g])
@@ -115,7 +131,7 @@ def forward(q, k, v, kd, vd, scale: float, row_block: int = 256):
     return out, lse
 
 
-def forward_rows(q, k, v, kd, vd, scale: float, b: int, h: int, ts):
+def forward_rows(q, k, v, kd, vd, scale: float, b: int, h: int, ts, depth_sel=None):
     """MoDA forward for selected positions ``ts`` of one (b, h).
 
     Same definition as ``forward``; used to check long sequences on sampled
@@ -131,14 +147,19 @@ def forward_rows(q, k, v, kd, vd, scale: float, b: int, h: int, ts):
     vseq = to_f64(v[b, :jmax, g])
     kdep = to_f64(kd[b][idx])[:, :, g]
     vdep = to_f64(vd[b][idx])[:, :, g]
-    s = _concat_logits(qr, kseq, kdep, scale, ts)
+    sel = None if depth_sel is None else np.asarray(depth_sel[b][idx], dtype=bool)
+    s = _concat_logits(qr, kseq, kdep, scale, ts, sel)
     p, l = _softmax_rows(s)
     vals = p[:, :jmax] @ vseq + np.einsum("ri,ric->rc", p[:, jmax:], vdep)
     return vals, l
 
 
-def backward(q, k, v, kd, vd, dout, scale: float, row_block: int = 256, out_for_D=None):
+def backward(q, k, v, kd, vd, dout, scale: float, row_block: int = 256, out_for_D=None,
+             depth_sel=None):
     """Gradients of the MoDA forward for upstream gradient ``dout``.
+
+    ``depth_sel`` (optional, [B,T,Ld] bool): as in ``forward``; unselected
+    depth entries get zero gradients.
 
     ``out_for_D`` (optional, [B,T,Hq,d]): the forward output to form
     D = <dout, out> from. By default D uses the exact float64 forward output,
@@ -161,7 +182,7 @@ def backward(q, k, v, kd, vd, dout, scale: float, row_block: int = 256, out_for_
     """
     q, k, v, kd, vd, dout = (to_f64(x) for x in (q, k, v, kd, vd, dout))
     B, T, Hq, Hkv, G, d, Ld = _dims(q, k, kd)
-    out, lse = forward(q, k, v, kd, vd, scale, row_block)
+    out, lse = forward(q, k, v, kd, vd, scale, row_block, depth_sel)
     outD = out if out_for_D is None else to_f64(out_for_D)
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
@@ -176,7 +197,8 @@ def backward(q, k, v, kd, vd, dout, scale: float, row_block: int = 256, out_for_
                 ts = np.arange(t0, t1)
                 qr = q[b, t0:t1, h]
                 dor = dout[b, t0:t1, h]
-                s = _concat_logits(qr, k[b, :t1, g], kd[b, t0:t1, :, g], scale, ts)
+                s = _concat_logits(qr, k[b, :t1, g], kd[b, t0:t1, :, g], scale, ts,
+                                   _sel(depth_sel, b, t0, t1))
                 P = np.exp(s - lse[b, h, t0:t1][:, None])
                 D = np.sum(dor * outD[b, t0:t1, h], axis=1)
                 dP_seq = dor @ v[b, :t1, g].T

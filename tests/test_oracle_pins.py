@@ -276,17 +276,17 @@ def test_planted_mistakes_are_caught(monkeypatch):
 
     mutants = {
         # causal mask dropped (token sees the future)
-        "no_causal": lambda qr, ks, kdp, sc, ts: np.concatenate(
+        "no_causal": lambda qr, ks, kdp, sc, ts, sel=None: np.concatenate(
             [sc * (qr @ ks.T), sc * np.einsum("rc,ric->ri", qr, kdp)], axis=1),
         # strict causal mask (self excluded)
-        "strict_causal": lambda qr, ks, kdp, sc, ts: np.concatenate(
+        "strict_causal": lambda qr, ks, kdp, sc, ts, sel=None: np.concatenate(
             [np.where(np.arange(ks.shape[0])[None] < np.asarray(ts)[:, None], sc * (qr @ ks.T), -np.inf),
              sc * np.einsum("rc,ric->ri", qr, kdp)], axis=1),
         # depth logits without the scale
-        "unscaled_depth": lambda qr, ks, kdp, sc, ts: np.concatenate(
+        "unscaled_depth": lambda qr, ks, kdp, sc, ts, sel=None: np.concatenate(
             [orig(qr, ks, kdp[:, :0], sc, ts), np.einsum("rc,ric->ri", qr, kdp)], axis=1),
         # depth logits with a flipped sign
-        "neg_depth": lambda qr, ks, kdp, sc, ts: np.concatenate(
+        "neg_depth": lambda qr, ks, kdp, sc, ts, sel=None: np.concatenate(
             [orig(qr, ks, kdp[:, :0], sc, ts), -sc * np.einsum("rc,ric->ri", qr, kdp)], axis=1),
     }
     for name, fn in mutants.items():
@@ -330,3 +330,94 @@ def test_backward_with_stored_output_shifts_by_the_D_error():
                 acc += math.exp(scale * float(qv @ x["kd"][0, t, i, 0]) - lse[0, h, t]) * x["kd"][0, t, i, 0]
             np.testing.assert_allclose(pert[0][0, t, h] - base[0][0, t, h], -scale * dD * acc,
                                        rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------- selected depth
+def test_selected_depth_reduces_to_slicing_and_special_cases():
+    """Selection of all entries = no selection; a selection of the first L'
+    entries of every token = the forward with kd, vd sliced to L'; an empty
+    selection = Ld = 0 (plain causal attention)."""
+    x, scale = rand_case(2, 13, 4, 2, 8, 6, seed=31, depth_std=2.0)
+    B, T, Ld = 2, 13, 6
+    base = om.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale)
+    allsel = np.ones((B, T, Ld), dtype=bool)
+    o, l = om.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, depth_sel=allsel)
+    np.testing.assert_array_equal(o, base[0])
+    first = np.zeros((B, T, Ld), dtype=bool)
+    first[:, :, :4] = True
+    o, l = om.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, depth_sel=first)
+    o2, l2 = om.forward(x["q"], x["k"], x["v"], x["kd"][:, :, :4], x["vd"][:, :, :4], scale)
+    np.testing.assert_allclose(o, o2, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l, l2, rtol=0, atol=1e-13)
+    o, l = om.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, depth_sel=np.zeros_like(first))
+    o3, l3 = om.forward(x["q"], x["k"], x["v"], x["kd"][:, :, :0], x["vd"][:, :, :0], scale)
+    np.testing.assert_allclose(o, o3, rtol=0, atol=1e-13)
+
+
+def _selected_depth_case():
+    x, scale = rand_case(1, 6, 4, 2, 3, 4, seed=32, depth_std=2.0)
+    rng = np.random.default_rng(7)
+    sel = rng.random((1, 6, 4)) < 0.5
+    return x, scale, sel
+
+
+def _check_selected_depth_brute_force():
+    x, scale, sel = _selected_depth_case()
+    o, l = om.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, depth_sel=sel)
+    for t in range(6):
+        keep = np.flatnonzero(sel[0, t])
+        sub = {n: x[n][:, :t + 1] for n in ("q", "k", "v")}
+        kd = np.zeros((1, t + 1, len(keep), 2, 3))
+        vd = np.zeros_like(kd)
+        kd[0, t] = x["kd"][0, t, keep]
+        vd[0, t] = x["vd"][0, t, keep]
+        bo, bl = brute_force(sub["q"], sub["k"], sub["v"], kd, vd, scale)
+        np.testing.assert_allclose(o[0, t], bo[0, t], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l[0, :, t], bl[0, :, t], rtol=0, atol=1e-12)
+
+
+def test_selected_depth_brute_force_and_gradients():
+    """Per-token random selection against the scalar brute force run on each
+    token's gathered depth entries; backward against central differences, and
+    unselected depth entries get exactly zero gradient."""
+    _check_selected_depth_brute_force()
+    x, scale, sel = _selected_depth_case()
+    g = om.backward(x["q"], x["k"], x["v"], x["kd"], x["vd"], x["dout"], scale, depth_sel=sel)
+    assert np.all(g[3][~sel] == 0) and np.all(g[4][~sel] == 0)
+    eps = 1e-6
+    for name, gi in (("q", 0), ("kd", 3), ("vd", 4), ("k", 1)):
+        base = x[name]
+        it = np.nditer(base, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            old = base[idx]
+            base[idx] = old + eps
+            lp = float(np.sum(om.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, depth_sel=sel)[0] * x["dout"]))
+            base[idx] = old - eps
+            lm = float(np.sum(om.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, depth_sel=sel)[0] * x["dout"]))
+            base[idx] = old
+            assert abs((lp - lm) / (2 * eps) - g[gi][idx]) < 1e-6 * max(1.0, abs(g[gi][idx])), (name, idx)
+
+
+def test_planted_selection_mistakes_are_caught(monkeypatch):
+    """A selection ignored, inverted or taken from the neighbouring token
+    fails the selection pins."""
+    def sel_pins_pass():
+        try:
+            test_selected_depth_reduces_to_slicing_and_special_cases()
+            _check_selected_depth_brute_force()
+            return True
+        except AssertionError:
+            return False
+
+    assert sel_pins_pass()
+    orig_sel = om._sel
+    mutants = {
+        "ignored": lambda ds, b, t0, t1: None,
+        "inverted": lambda ds, b, t0, t1: None if ds is None else ~np.asarray(ds[b, t0:t1], dtype=bool),
+        "shifted": lambda ds, b, t0, t1: None if ds is None else np.roll(np.asarray(ds[b], dtype=bool), 1, axis=0)[t0:t1],
+    }
+    for name, fn in mutants.items():
+        monkeypatch.setattr(om, "_sel", fn)
+        assert not sel_pins_pass(), name
+        monkeypatch.setattr(om, "_sel", orig_sel)
