@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "MODA_OK", "ModaError", "lib", "LIB_PATH", "moda_abi_version", "moda_status_string",
-    "moda_fwd", "moda_bwd", "moda_bwd_workspace_bytes", "moda_bwd_noalloc", "moda_pack_depth",
+    "moda_fwd", "moda_fwd_sel", "moda_bwd", "moda_bwd_sel", "moda_bwd_workspace_bytes", "moda_bwd_noalloc", "moda_pack_depth",
     "moda_pack_depth_bytes", "moda_fwd_packed", "moda_device_status",
     "moda_debug_set_wait_limit", "moda_debug_exp2_poly", "moda_fwd_from_host",
 ]
@@ -49,9 +49,11 @@ _c_abi_version = _sig("moda_abi_version", _i, [])
 _c_status_string = _sig("moda_status_string", ctypes.c_char_p, [_i])
 _c_fwd_ex = _sig("moda_fwd_ex", _i, [_vp] * 5 + _DIMS + [_i, _f, _vp, _vp, _vp, _i])
 _c_fwd = _sig("moda_fwd", _i, [_vp] * 5 + _DIMS + [_i, _f, _vp, _vp, _vp])
+_c_fwd_sel = _sig("moda_fwd_sel", _i, [_vp] * 6 + _DIMS + [_i, _f, _vp, _vp, _vp, _i])
 _c_bwd_ws = _sig("moda_bwd_workspace_bytes", _sz, _DIMS + [_i])
 _c_bwd_ex = _sig("moda_bwd_ex", _i, [_vp] * 8 + _DIMS + [_i, _f] + [_vp] * 5 + [_vp, _sz, _vp, _i])
 _c_bwd = _sig("moda_bwd", _i, [_vp] * 8 + _DIMS + [_i, _f] + [_vp] * 5 + [_vp, _sz, _vp])
+_c_bwd_sel = _sig("moda_bwd_sel", _i, [_vp] * 9 + _DIMS + [_i, _f] + [_vp] * 5 + [_vp, _sz, _vp, _i])
 _c_pack_bytes = _sig("moda_pack_depth_bytes", _sz, [_i] * 5 + [_i])
 _c_pack = _sig("moda_pack_depth", _i, [_vp, _vp] + [_i] * 5 + [_i, _vp, _vp])
 _c_fwd_packed = _sig("moda_fwd_packed", _i, [_vp] * 4 + _DIMS + [_i, _f, _vp, _vp, _vp])
@@ -129,6 +131,59 @@ def moda_fwd(q, k, v, kd=None, vd=None, scale: float | None = None, out=None, ls
                          _DTYPE[q.dtype], scale, _ptr(out), _ptr(lse), _stream(stream), _IMPL[impl]),
                "moda_fwd")
     return out, lse
+
+
+def _check_sel(depth_sel, B, T):
+    if depth_sel is None:
+        return
+    if depth_sel.dtype != torch.int64 or tuple(depth_sel.shape) != (B, T):
+        raise ValueError("depth_sel must be an int64 [B, T] tensor of depth-slot bit masks")
+
+
+def moda_fwd_sel(q, k, v, kd, vd, depth_sel, scale: float | None = None, out=None, lse=None,
+                 impl: str = "auto", stream=None):
+    """MoDA forward with per-token depth-slot selection (``moda_fwd_sel``).
+
+    ``depth_sel``: int64 [B, T] bit masks (bit i set = the token's depth slot
+    i takes part), or None for every slot. Returns (out, lse)."""
+    _check_tensors(q, k, v, kd, vd, depth_sel, out, lse)
+    B, T, Hq, Hkv, d, Ld = _dims(q, k, kd)
+    _check_sel(depth_sel, B, T)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
+    with torch.cuda.device(q.device):
+        _check(_c_fwd_sel(_ptr(q), _ptr(k), _ptr(v), _ptr(kd), _ptr(vd), _ptr(depth_sel), B, T, Hq,
+                          Hkv, d, Ld, _DTYPE[q.dtype], scale, _ptr(out), _ptr(lse), _stream(stream),
+                          _IMPL[impl]), "moda_fwd_sel")
+    return out, lse
+
+
+def moda_bwd_sel(q, k, v, kd, vd, depth_sel, out, lse, dout, scale: float | None = None,
+                 grads=None, workspace=None, impl: str = "auto", stream=None):
+    """Gradients of ``moda_fwd_sel`` (``moda_bwd_sel``), same ``depth_sel``.
+    Returns (dq, dk, dv, dkd, dvd)."""
+    _check_tensors(q, k, v, kd, vd, depth_sel, out, lse, dout)
+    B, T, Hq, Hkv, d, Ld = _dims(q, k, kd)
+    _check_sel(depth_sel, B, T)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                 torch.empty_like(kd), torch.empty_like(vd))
+    dq, dk, dv, dkd, dvd = grads
+    need = moda_bwd_workspace_bytes(B, T, Hq, Hkv, d, Ld, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    with torch.cuda.device(q.device):
+        _check(_c_bwd_sel(_ptr(q), _ptr(k), _ptr(v), _ptr(kd), _ptr(vd), _ptr(depth_sel), _ptr(out),
+                          _ptr(lse), _ptr(dout), B, T, Hq, Hkv, d, Ld, _DTYPE[q.dtype], scale,
+                          _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dkd), _ptr(dvd), _ptr(workspace),
+                          workspace.numel(), _stream(stream), _IMPL[impl]), "moda_bwd_sel")
+    return dq, dk, dv, dkd, dvd
 
 
 def moda_bwd_workspace_bytes(B, T, Hq, Hkv, d, Ld, dtype) -> int:

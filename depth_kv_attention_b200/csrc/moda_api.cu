@@ -71,6 +71,15 @@ moda_status fill_fwd(FwdArgs& a, const void* q, const void* k, const void* v, co
     return MODA_OK;
 }
 
+// Depth-slot masks: 8-byte aligned, one 64-bit word per token, so Ld <= 64.
+moda_status set_sel(FwdArgs& a, const uint64_t* depth_sel) {
+    if (!depth_sel) return MODA_OK;
+    if ((reinterpret_cast<uintptr_t>(depth_sel) & 7u) != 0) return MODA_ERR_MISALIGNED;
+    if (a.Ld > 64) return MODA_ERR_UNSUPPORTED;
+    a.depth_sel = reinterpret_cast<const unsigned long long*>(depth_sel);
+    return MODA_OK;
+}
+
 moda_status run_fwd(FwdArgs& a, void* stream, moda_impl impl) {
     cudaError_t e = status_ptr(&a.status, &a.wait_limit);
     if (e != cudaSuccess) return MODA_ERR_CUDA;
@@ -115,15 +124,25 @@ const char* moda_status_string(moda_status s) {
     return "MODA_ERR_UNKNOWN";
 }
 
-moda_status moda_fwd_ex(const void* q, const void* k, const void* v, const void* kd, const void* vd,
-                        int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dtype, float scale,
-                        void* out, float* lse, void* stream, moda_impl impl) {
+moda_status moda_fwd_sel(const void* q, const void* k, const void* v, const void* kd,
+                         const void* vd, const uint64_t* depth_sel, int B, int T, int Hq, int Hkv,
+                         int d, int Ld, moda_dtype dtype, float scale, void* out, float* lse,
+                         void* stream, moda_impl impl) {
     if (impl != MODA_IMPL_AUTO && impl != MODA_IMPL_SIMT && impl != MODA_IMPL_TC)
         return MODA_ERR_INVALID_VALUE;
     FwdArgs a;
     moda_status st = fill_fwd(a, q, k, v, kd, vd, B, T, Hq, Hkv, d, Ld, dtype, scale, out, lse, false);
     if (st != MODA_OK) return st;
+    st = set_sel(a, depth_sel);
+    if (st != MODA_OK) return st;
     return run_fwd(a, stream, impl);
+}
+
+moda_status moda_fwd_ex(const void* q, const void* k, const void* v, const void* kd, const void* vd,
+                        int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dtype, float scale,
+                        void* out, float* lse, void* stream, moda_impl impl) {
+    return moda_fwd_sel(q, k, v, kd, vd, nullptr, B, T, Hq, Hkv, d, Ld, dtype, scale, out, lse,
+                        stream, impl);
 }
 
 moda_status moda_fwd(const void* q, const void* k, const void* v, const void* kd, const void* vd,
@@ -141,17 +160,20 @@ size_t moda_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int Ld, mo
     return bwd_ws_bytes(B, T, Hq, Hkv, d, dtype == MODA_BF16);
 }
 
-moda_status moda_bwd_ex(const void* q, const void* k, const void* v, const void* kd, const void* vd,
-                        const void* out, const float* lse, const void* dout, int B, int T, int Hq,
-                        int Hkv, int d, int Ld, moda_dtype dtype, float scale, void* dq, void* dk,
-                        void* dv, void* dkd, void* dvd, void* workspace, size_t workspace_bytes,
-                        void* stream, moda_impl impl) {
+moda_status moda_bwd_sel(const void* q, const void* k, const void* v, const void* kd,
+                         const void* vd, const uint64_t* depth_sel, const void* out,
+                         const float* lse, const void* dout, int B, int T, int Hq, int Hkv, int d,
+                         int Ld, moda_dtype dtype, float scale, void* dq, void* dk, void* dv,
+                         void* dkd, void* dvd, void* workspace, size_t workspace_bytes,
+                         void* stream, moda_impl impl) {
     if (impl != MODA_IMPL_AUTO && impl != MODA_IMPL_SIMT && impl != MODA_IMPL_TC)
         return MODA_ERR_INVALID_VALUE;
     BwdArgs a;
     std::memset(&a, 0, sizeof(a));
     moda_status st = fill_fwd(a.f, q, k, v, kd, vd, B, T, Hq, Hkv, d, Ld, dtype, scale,
                               const_cast<void*>(out), const_cast<float*>(lse), false);
+    if (st != MODA_OK) return st;
+    st = set_sel(a.f, depth_sel);
     if (st != MODA_OK) return st;
     if (!lse || !dout || !dq || !dk || !dv) return MODA_ERR_INVALID_VALUE;
     if (Ld > 0 && (!dkd || !dvd)) return MODA_ERR_INVALID_VALUE;
@@ -176,6 +198,15 @@ moda_status moda_bwd_ex(const void* q, const void* k, const void* v, const void*
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     e = use_tc ? launch_bwd_tc(a, s) : launch_bwd_simt(a, s);
     return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
+}
+
+moda_status moda_bwd_ex(const void* q, const void* k, const void* v, const void* kd, const void* vd,
+                        const void* out, const float* lse, const void* dout, int B, int T, int Hq,
+                        int Hkv, int d, int Ld, moda_dtype dtype, float scale, void* dq, void* dk,
+                        void* dv, void* dkd, void* dvd, void* workspace, size_t workspace_bytes,
+                        void* stream, moda_impl impl) {
+    return moda_bwd_sel(q, k, v, kd, vd, nullptr, out, lse, dout, B, T, Hq, Hkv, d, Ld, dtype,
+                        scale, dq, dk, dv, dkd, dvd, workspace, workspace_bytes, stream, impl);
 }
 
 moda_status moda_bwd(const void* q, const void* k, const void* v, const void* kd, const void* vd,

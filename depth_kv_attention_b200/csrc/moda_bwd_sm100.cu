@@ -31,6 +31,7 @@
 #include <cmath>
 #include <cstring>
 
+#include "depth_mask.cuh"
 #include "moda_internal.h"
 #include "sm100_ptx.cuh"
 #include "tmap_host.h"
@@ -129,6 +130,7 @@ struct DkvParams {
     void* dkd;      // depth mode: [B,T,Ld,Hkv,d] bf16 outputs
     void* dvd;
     int depth_mode, Ld;
+    const unsigned long long* depth_sel;  // depth mode: [B,T] slot masks or null
     int B, T, Hq, Hkv, G, n, gshift, qchunk;
     float sl2, scale;
     unsigned int* status;
@@ -278,6 +280,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
         const int r = warp * 32 + lane;  // TMEM lane
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const int j = j0 + r;            // this thread's key
+        // depth mode: is depth row j (slot j % Ld of token j / Ld) selected?
+        const bool j_selected = !p.depth_mode || !p.depth_sel || j >= p.T * p.Ld ||
+                                ((p.depth_sel[(long long)b * p.T + j / p.Ld] >> (j % p.Ld)) & 1ull);
         const float sl2 = p.sl2;
         const int gshift = p.gshift;
         bool ok = true;
@@ -318,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
             if (p.depth_mode) {
                 const int td = j < p.T * p.Ld ? j / p.Ld : -1;
                 lo_r = (td - tq0) * p.G;
-                hi_r = td < 0 ? lo_r : lo_r + p.G;
+                hi_r = (td < 0 || !j_selected) ? lo_r : lo_r + p.G;
             } else {
                 lo_r = j > tq0 ? (j - tq0) << gshift : 0;
                 hi_r = 128;
@@ -433,6 +438,7 @@ struct DqParams {
     const float* lse;
     const float* rowD;
     void* dq;  // [B,T,Hq,d] bf16
+    const unsigned long long* depth_sel;  // [B,T] slot masks or null
     int B, T, Hq, Hkv, G, n, Ld, nqt;
     float sl2, scale;
     unsigned int* status;
@@ -608,6 +614,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
             Drow = p.rowD[ix];
         }
         const float sl2 = p.sl2;
+        const bool has_sel = p.depth_sel != nullptr;
+        const unsigned long long sel =
+            has_sel && row_ok ? p.depth_sel[(long long)b * p.T + t] & depth_slot_bits(p.Ld) : 0ull;
         bool ok = true;
         for (int x = 0; x < n_items; ++x) {
             const uint32_t rS = tmem + lane_off + (x & 1) * 128;        // S(x), then dS(x)
@@ -624,21 +633,18 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
 #pragma unroll
                 for (int c = 0; c < 4; ++c) ptx::tmem_ld32(rS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&su[c * 32]));
                 ptx::tmem_wait_ld();
-                int lo, hi;  // visible columns of this row
-                if (x < n_kv) {
-                    lo = 0;
-                    hi = t - x * kBK + 1;  // keys <= t
-                } else {
-                    lo = tt * p.Ld - (x - n_kv) * kBK;  // the row's own depth rows
-                    hi = lo + p.Ld;
-                }
+                uint32_t vis[4];  // visible columns of this row
+                if (x < n_kv)
+                    depth_col_mask(0, t - x * kBK + 1, false, 0ull, vis);  // keys <= t
+                else  // the row's own depth rows (selected slots)
+                    depth_col_mask(tt * p.Ld - (x - n_kv) * kBK, p.Ld, has_sel, sel, vis);
 #pragma unroll
                 for (int c = 0; c < 128; c += 2) {
                     const float2 e = exp2_pair(make_float2(fmaf(__uint_as_float(su[c]), sl2, -lse2),
                                                            fmaf(__uint_as_float(su[c + 1]), sl2, -lse2)),
                                                c / 2);
-                    pr[c] = (c >= lo && c < hi) ? e.x : 0.f;
-                    pr[c + 1] = (c + 1 >= lo && c + 1 < hi) ? e.y : 0.f;
+                    pr[c] = ((vis[c >> 5] >> (c & 31)) & 1u) ? e.x : 0.f;
+                    pr[c + 1] = ((vis[c >> 5] >> ((c + 1) & 31)) & 1u) ? e.y : 0.f;
                 }
             }
             if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->dp_full, x & 1, p.wait_limit, abort_flag))) {
@@ -802,6 +808,7 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s) {
         pd.tm_v = tm_vd;
         pd.depth_mode = 1;
         pd.Ld = f.Ld;
+        pd.depth_sel = f.depth_sel;
         pd.dkd = a.dkd;
         pd.dvd = a.dvd;
         const long long chunks = ((long long)f.T * f.Ld + kBK - 1) / kBK;
@@ -817,6 +824,7 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s) {
     pq.lse = f.lse; pq.rowD = a.rowD; pq.dq = a.dq;
     pq.B = f.B; pq.T = f.T; pq.Hq = f.Hq; pq.Hkv = f.Hkv; pq.G = G; pq.n = n; pq.Ld = f.Ld;
     pq.nqt = (f.T + n - 1) / n;
+    pq.depth_sel = f.depth_sel;
     pq.sl2 = f.scale * kLog2e; pq.scale = f.scale;
     pq.status = f.status; pq.wait_limit = f.wait_limit;
     if ((e = cudaFuncSetAttribute(moda_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem)) !=

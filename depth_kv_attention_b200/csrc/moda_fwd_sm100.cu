@@ -38,6 +38,7 @@
 #include <cmath>
 #include <cstring>
 
+#include "depth_mask.cuh"
 #include "moda_internal.h"
 #include "sm100_ptx.cuh"
 #include "tmap_host.h"
@@ -82,6 +83,7 @@ struct TcFwdParams {
     int B, T, Hq, Hkv, G, n, Ld, nblk;
     float sl2;  // scale * log2(e)
     int depth_packed;
+    const unsigned long long* depth_sel;  // [B,T] slot masks or null
     unsigned int* status;
     unsigned int wait_limit;
 };
@@ -336,6 +338,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
         const int t = t0 + tl;
         const int h = kvh * p.G + r % p.G;
         const float sl2 = p.sl2;
+        const bool has_sel = p.depth_sel != nullptr;
+        const unsigned long long sel =
+            has_sel && t < p.T ? p.depth_sel[(long long)b * p.T + t] & depth_slot_bits(p.Ld) : 0ull;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         int it = 0;                        // items this tile has taken part in
@@ -369,12 +374,12 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                 }
             } else {
                 // same-token mask: this row's depth rows are [tl*Ld, (tl+1)*Ld)
-                // of the unit's depth range
-                const int lo = tl * p.Ld - (x - n_seq) * kBN;
-                const int hi = lo + p.Ld;
+                // of the unit's depth range (selected slots only)
+                uint32_t vis[4];
+                depth_col_mask(tl * p.Ld - (x - n_seq) * kBN, p.Ld, has_sel, sel, vis);
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
-                    if (c < lo || c >= hi) s[c] = -INFINITY;
+                    if (!((vis[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
             }
             float mx;
             {
@@ -566,6 +571,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s) {
     p.nblk = (a.T + 2 * n - 1) / (2 * n);
     p.sl2 = a.scale * 1.4426950408889634f;
     p.depth_packed = packed ? 1 : 0;
+    p.depth_sel = a.depth_sel;
     p.status = a.status;
     p.wait_limit = a.wait_limit;
     cudaError_t err = cudaFuncSetAttribute(moda_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);

@@ -33,6 +33,7 @@ struct FwdArgs {
     Strides4 sq, skv, so;
     Strides5 sdep;    // kd and vd share strides
     moda_dtype dtype;
+    const unsigned long long* depth_sel;  // [B,T] depth-slot bit masks, or null (all slots)
     unsigned int* status;     // device status word
     unsigned int wait_limit;  // bounded-wait polls (0 = kernel default)
 };

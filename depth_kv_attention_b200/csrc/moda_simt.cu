@@ -161,12 +161,17 @@ __global__ void __launch_bounds__(128) fwd_simt_kernel(FwdArgs a, int n_tok, int
     for (int i = 0; i < S::NP; ++i) o[i] = make_float2(0.f, 0.f);
     float m = -INFINITY, l = 0.f;
 
-    // Depth keys of the same token (depth mask): read straight from global.
+    // Depth keys of the same token (depth mask), of the slots the token
+    // selects: read straight from global. Rows of one warp select different
+    // slots, so every lane runs the shuffles of group_sum and an unselected
+    // slot is skipped only after them.
+    const unsigned long long sel = a.depth_sel ? a.depth_sel[(long long)b * a.T + tc] : 0ull;
     for (int i = 0; i < a.Ld; ++i) {
         const long long off = b * a.sdep.sb + tc * a.sdep.st + (long long)i * a.sdep.si + kvh * a.sdep.sh;
         float2 kr[S::NP];
         load_row<TPR>(KD + off, a.d, u, kr);
         const float s = group_sum<TPR>(dot_regs<TPR>(q, kr));
+        if (a.depth_sel && !((sel >> i) & 1ull)) continue;
         float2 vr[S::NP];
         load_row<TPR>(VD + off, a.d, u, vr);
         if (s > m) {
@@ -263,7 +268,9 @@ __global__ void __launch_bounds__(256) bwd_dq_simt_kernel(BwdArgs a, int n_tok, 
     const float lse2 = f.lse[rix] * kLog2e;
     const float Drow = a.rowD[rix];
 
-    // Depth part: dq += dS'_i kd_i.
+    // Depth part: dq += dS'_i kd_i over the selected slots (skipped only
+    // after the warp-wide shuffles of group_sum, as in the forward).
+    const unsigned long long sel = f.depth_sel ? f.depth_sel[(long long)b * f.T + tc] : 0ull;
     for (int i = 0; i < f.Ld; ++i) {
         const long long off = b * f.sdep.sb + tc * f.sdep.st + (long long)i * f.sdep.si + kvh * f.sdep.sh;
         float2 kr[S::NP], vr[S::NP];
@@ -271,6 +278,7 @@ __global__ void __launch_bounds__(256) bwd_dq_simt_kernel(BwdArgs a, int n_tok, 
         load_row<TPR>(static_cast<const T*>(f.vd) + off, f.d, u, vr);
         const float s = group_sum<TPR>(dot_regs<TPR>(q, kr));
         const float dp = group_sum<TPR>(dot_regs<TPR>(dO, vr));
+        if (f.depth_sel && !((sel >> i) & 1ull)) continue;
         const float p = exp2f(s - lse2);
         axpy_regs<TPR>(dq, p * (dp - Drow), kr);
     }
@@ -385,6 +393,10 @@ __global__ void __launch_bounds__(256) bwd_depth_simt_kernel(BwdArgs a) {
     load_row<TPR>(static_cast<const T*>(f.vd) + off, f.d, u, vd);
 #pragma unroll
     for (int c = 0; c < S::NP; ++c) { dkd[c] = make_float2(0.f, 0.f); dvd[c] = make_float2(0.f, 0.f); }
+    // An unselected slot is absent from every row: zero gradients (its
+    // probabilities are zeroed; the loop itself stays warp-uniform because
+    // group_sum shuffles across the whole warp).
+    const bool selected = !f.depth_sel || ((f.depth_sel[(long long)b * f.T + t] >> i) & 1ull);
     for (int g = 0; g < f.G; ++g) {
         const int h = kvh * f.G + g;
         float2 q[S::NP], dO[S::NP];
@@ -393,7 +405,7 @@ __global__ void __launch_bounds__(256) bwd_depth_simt_kernel(BwdArgs a) {
         const long long rix = ((long long)b * f.Hq + h) * f.T + t;
         const float s = group_sum<TPR>(dot_regs<TPR>(q, kd));
         const float dp = group_sum<TPR>(dot_regs<TPR>(dO, vd));
-        const float p = exp2f(s - f.lse[rix] * kLog2e);
+        const float p = selected ? exp2f(s - f.lse[rix] * kLog2e) : 0.f;
         axpy_regs<TPR>(dvd, p, dO);
         axpy_regs<TPR>(dkd, p * (dp - a.rowD[rix]), q);
     }

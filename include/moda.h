@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define MODA_ABI_VERSION 1
+#define MODA_ABI_VERSION 2
 
 typedef enum {
     MODA_OK = 0,
@@ -112,6 +112,29 @@ moda_status moda_fwd_ex(const void* q, const void* k, const void* v,
                         void* out, float* lse, void* stream, moda_impl impl);
 
 /*
+ * moda_fwd_sel — moda_fwd with a per-token selection of depth slots: the
+ * bounded depth-KV slots ("sliding window" over layers or a dynamic choice of
+ * layers) that "Mixture-of-Depths Attention" (gist.science German summary §5,
+ * future directions) proposes for very deep models.
+ *   depth_sel [B,T] uint64  in  device bit masks, 8-byte aligned: bit i of
+ *                               depth_sel[b*T + t] set = token t's depth slot
+ *                               i (kd[b,t,i], vd[b,t,i]) takes part in its
+ *                               softmax; clear = that slot is absent for
+ *                               every head of the token. Bits >= Ld are
+ *                               ignored. NULL = every slot (= moda_fwd_ex).
+ * A token whose mask is 0 attends to its causal sequence keys only (its own
+ * key is always visible, so no row is empty). A non-NULL mask needs
+ * Ld <= 64, else MODA_ERR_UNSUPPORTED. The depth keys of unselected slots are
+ * still read (the kernels load whole tiles); only the result changes.
+ * Other arguments, semantics and errors as moda_fwd_ex.
+ */
+moda_status moda_fwd_sel(const void* q, const void* k, const void* v,
+                         const void* kd, const void* vd, const uint64_t* depth_sel,
+                         int B, int T, int Hq, int Hkv, int d, int Ld,
+                         moda_dtype dtype, float scale,
+                         void* out, float* lse, void* stream, moda_impl impl);
+
+/*
  * moda_bwd_workspace_bytes — bytes of fp32 scratch moda_bwd needs for this
  * shape: row statistics D [B,Hq,T] and, for bf16 (tensor-core path), fp32
  * accumulators of dk and dv [B,T,Hkv,d]. Returns 0 for an invalid shape.
@@ -151,6 +174,21 @@ moda_status moda_bwd_ex(const void* q, const void* k, const void* v,
                         void* dq, void* dk, void* dv, void* dkd, void* dvd,
                         void* workspace, size_t workspace_bytes, void* stream,
                         moda_impl impl);
+
+/*
+ * moda_bwd_sel — gradients of moda_fwd_sel: moda_bwd_ex with the same
+ * depth_sel as the forward (out and lse must come from moda_fwd_sel with that
+ * mask). Unselected depth slots get dkd = dvd = 0; the other gradients see
+ * only the selected slots. depth_sel NULL = moda_bwd_ex.
+ */
+moda_status moda_bwd_sel(const void* q, const void* k, const void* v,
+                         const void* kd, const void* vd, const uint64_t* depth_sel,
+                         const void* out, const float* lse, const void* dout,
+                         int B, int T, int Hq, int Hkv, int d, int Ld,
+                         moda_dtype dtype, float scale,
+                         void* dq, void* dk, void* dv, void* dkd, void* dvd,
+                         void* workspace, size_t workspace_bytes, void* stream,
+                         moda_impl impl);
 
 /*
  * moda_bwd_noalloc — moda_bwd for callers that cannot allocate device memory.

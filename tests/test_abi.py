@@ -23,7 +23,7 @@ def declared_functions():
 
 def test_header_declares_the_abi():
     fns = declared_functions()
-    for name in ["moda_fwd", "moda_bwd", "moda_bwd_workspace_bytes", "moda_pack_depth",
+    for name in ["moda_fwd", "moda_fwd_sel", "moda_bwd", "moda_bwd_sel", "moda_bwd_workspace_bytes", "moda_pack_depth",
                  "moda_fwd_packed", "moda_device_status", "moda_status_string"]:
         assert name in fns
 
@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_status_strings():
-    assert moda.moda_abi_version() == 1
+    assert moda.moda_abi_version() == 2
     assert moda.moda_status_string(0) == "MODA_OK"
     assert moda.moda_status_string(6) == "MODA_ERR_DEVICE_TIMEOUT"
     assert moda.moda_status_string(99) == "MODA_ERR_UNKNOWN"
@@ -86,3 +86,24 @@ def test_workspace_and_pack_sizes():
     assert moda._c_pack_bytes(2, 5, 3, 128, 7, 0) == 2 * 2 * 5 * 7 * 3 * 128 * 2
     assert moda._c_pack(P, P, 1, 4, 1, 128, 2, 0, P + 8, None) == 3
     assert moda._c_pack(P, P, 1, 4, 1, 6, 2, 0, P, None) == 2
+
+
+def fwd_sel(sel=P, Ld=2, d=64, q=P):
+    return moda._c_fwd_sel(q, P, P, P, P, sel, 1, 8, 4, 2, d, Ld, 0, 0.125, P, P, None, 0)
+
+
+def bwd_sel(sel=P, Ld=2, dq=P):
+    return moda._c_bwd_sel(P, P, P, P, P, sel, P, P, P, 1, 8, 4, 2, 64, Ld, 0, 0.125, dq, P, P, P, P,
+                           P, 1 << 30, None, 0)
+
+
+def test_selection_validation():
+    """Depth-slot masks: 8-byte aligned, at most 64 slots; the checks of the
+    unselected entry points still apply."""
+    assert fwd_sel(sel=P + 4) == 3
+    assert fwd_sel(Ld=65) == 2
+    assert fwd_sel(d=0) == 1
+    assert fwd_sel(q=P + 2) == 3
+    assert bwd_sel(sel=P + 4) == 3
+    assert bwd_sel(Ld=65) == 2
+    assert bwd_sel(dq=None) == 1
