@@ -27,7 +27,7 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from moda_inputs import WORKLOADS, make_inputs, sample_rows  # noqa: E402
+from moda_inputs import WORKLOADS, make_depth_sel, make_inputs, pack_depth_sel, sample_rows  # noqa: E402
 
 METRIC = "MoDA fwd TFLOP/s at T=64K (1×B200), % BF16 peak, overhead vs Ld=0 attention"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -238,13 +238,20 @@ def workload_config(w):
             "parallelism": "replicas"}
 
 
-def make_step(moda, w, x, mode, kernel):
+def make_step(moda, w, x, mode, kernel, depth_sel=None):
     """The timed step on device-resident inputs: one forward, or forward and
-    backward. Returns (step, launches of this library's kernels per step,
-    out, lse)."""
+    backward; with ``depth_sel`` (int64 [B, T] slot masks on the device) the
+    selected-depth entry points. Returns (step, launches of this library's
+    kernels per step, out, lse)."""
     out = torch.empty_like(x["q"])
     lse = torch.empty((w.B, w.Hq, w.T), device="cuda", dtype=torch.float32)
     if mode == "fwd":
+        if depth_sel is not None:
+            def step():
+                moda.moda_fwd_sel(x["q"], x["k"], x["v"], x["kd"], x["vd"], depth_sel, w.scale,
+                                  out=out, lse=lse, impl=kernel)
+            return step, 1, out, lse
+
         def step():
             moda.moda_fwd(x["q"], x["k"], x["v"], x["kd"], x["vd"], w.scale, out=out, lse=lse,
                           impl=kernel)
@@ -256,6 +263,12 @@ def make_step(moda, w, x, mode, kernel):
                      device="cuda", dtype=torch.uint8)
 
     def step():
+        if depth_sel is not None:
+            moda.moda_fwd_sel(x["q"], x["k"], x["v"], x["kd"], x["vd"], depth_sel, w.scale,
+                              out=out, lse=lse, impl=kernel)
+            moda.moda_bwd_sel(x["q"], x["k"], x["v"], x["kd"], x["vd"], depth_sel, out, lse,
+                              x["dout"], w.scale, grads=grads, workspace=ws, impl=kernel)
+            return
         moda.moda_fwd(x["q"], x["k"], x["v"], x["kd"], x["vd"], w.scale, out=out, lse=lse,
                       impl=kernel)
         moda.moda_bwd(x["q"], x["k"], x["v"], x["kd"], x["vd"], out, lse, x["dout"], w.scale,
@@ -277,12 +290,23 @@ def measure_secondary(moda, w, world, kernel, steps=5, warmup=3):
     res = {"config": f"B={w.B} T={w.T} Hq={w.Hq} Hkv={w.Hkv} d={w.d} Ld={w.Ld}",
            "fwd_ms": ms, "fwd_tflops": credited_flops(w) / (ms * 1e-3) / 1e12,
            "ld0_fwd_ms": ms0, "overhead_vs_ld0": ms / ms0 - 1.0}
+    # Selected depth: each token keeps a window of its most recent slots
+    # (width uniform in [0, Ld]), the same FLOPs are issued (whole tiles).
+    sel = pack_depth_sel(make_depth_sel(w, "window")).cuda() if w.Ld else None
+    if sel is not None:
+        steps_sel, _, _, _ = make_step(moda, w, x, "fwd", kernel, depth_sel=sel)
+        mss, _ = timed(steps_sel, steps, warmup, world)
+        res.update({"sel_window_fwd_ms": mss, "sel_vs_all_slots": mss / ms - 1.0})
     if w.backward:
         stepb, _, _, _ = make_step(moda, w, x, "fwdbwd", kernel)
         msb, _ = timed(stepb, steps, warmup, world)
         res.update({"fwd_bwd_ms": msb, "bwd_ms": msb - ms,
                     "bwd_tflops": 2.5 * credited_flops(w) / ((msb - ms) * 1e-3) / 1e12,
                     "fwd_bwd_tflops": 3.5 * credited_flops(w) / (msb * 1e-3) / 1e12})
+        if sel is not None:
+            stepbs, _, _, _ = make_step(moda, w, x, "fwdbwd", kernel, depth_sel=sel)
+            msbs, _ = timed(stepbs, steps, warmup, world)
+            res.update({"sel_window_fwd_bwd_ms": msbs, "sel_fwd_bwd_vs_all_slots": msbs / msb - 1.0})
     del x
     torch.cuda.empty_cache()
     return res
