@@ -43,9 +43,12 @@ constexpr int kD = 128;
 constexpr int kBK = 128;          // keys per key tile
 constexpr int kTile = 128 * kD * 2;
 constexpr int kHalf = kTile / 2;
-constexpr int kThreads = 192;     // warps 0-3 compute, 4 TMA producer, 5 MMA
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+// Warps 0-7 compute (two warpgroups: column halves 0-63 and 64-127 of every
+// TMEM tile; warp w reaches TMEM lanes 32*(w%4) ..), 8 TMA producer, 9 MMA.
+constexpr int kThreads = 320;
+constexpr int kComputeThreads = 256;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr float kLog2e = 1.4426950408889634f;
 // Of every 8 column pairs, pairs kBwdPolyFrom..7 take exp2 from the FMA-pipe
 // polynomial, the rest from MUFU (in these kernels the exponentials sit on
@@ -70,25 +73,29 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
 }
-// Barrier 1 spans the 128 compute threads only.
-__device__ __forceinline__ void named_sync_compute() {
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+// Barrier 1 + hs spans the 128 compute threads of column half hs only.
+__device__ __forceinline__ void half_sync(int hs) {
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + hs) : "memory");
 }
-// AND of `v` over the 128 compute threads (a barrier too): every compute
-// warp takes the same branch after a bounded wait, so none is left waiting at
-// a later named barrier.
-__device__ __forceinline__ bool all_compute(bool v) {
+// AND of `v` over the 128 compute threads of column half hs (a barrier too):
+// every warp of the half takes the same branch after a bounded wait, so none
+// is left waiting at a later named barrier.
+__device__ __forceinline__ bool half_all(int hs, bool v) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred pi, po;\n\t"
         "setp.ne.u32 pi, %1, 0;\n\t"
-        "bar.red.and.pred po, 1, 128, pi;\n\t"
+        "bar.red.and.pred po, %2, 128, pi;\n\t"
         "selp.u32 %0, 1, 0, po;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)v)
+        : "r"((uint32_t)v), "r"(1 + hs)
         : "memory");
     return r != 0;
 }
+// TMEM column of K step k (16 rows of the reduced dimension = 8 packed
+// columns) of a bf16 A operand whose two column halves each wrote their
+// packed values at the start of their own 64 columns.
+__device__ __forceinline__ uint32_t acol(int k) { return (uint32_t)((k >> 2) * 64 + (k & 3) * 8); }
 
 struct __align__(8) Bars {
     uint64_t kv_full;            // dk/dv kernel: K, V tile | dq kernel: Q, dO tile
@@ -112,7 +119,7 @@ __device__ __forceinline__ void init_bars(Bars* bars, int stages) {
     }
     ptx::mbar_init(&bars->s_full, 1);
     ptx::mbar_init(&bars->dp_full, 1);
-    ptx::mbar_init(&bars->p_full, 128);
+    ptx::mbar_init(&bars->p_full, kComputeThreads);
     ptx::mbar_init(&bars->fin, 1);
     ptx::mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -265,10 +272,10 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
             ptx::tc_fence_after();
 #pragma unroll
             for (int k = 0; k < 128 / 16; ++k)
-                ptx::mma_ts_lead(tmem + 256, tmem + 0 + k * 8, dOm + mnoff(k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u, lead);
+                ptx::mma_ts_lead(tmem + 256, tmem + 0 + acol(k), dOm + mnoff(k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u, lead);
 #pragma unroll
             for (int k = 0; k < 128 / 16; ++k)
-                ptx::mma_ts_lead(tmem + 384, tmem + 128 + k * 8, dQm + mnoff(k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u, lead);
+                ptx::mma_ts_lead(tmem + 384, tmem + 128 + acol(k), dQm + mnoff(k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u, lead);
             ptx::mma_commit_lead(&bars->empty[st], lead);
         }
         if (ok) ptx::mma_commit_lead(&bars->fin, lead);
@@ -277,8 +284,11 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
         __syncwarp();
     } else {
         // ------------------------------------------------------ compute warps
-        const int r = warp * 32 + lane;  // TMEM lane
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // Column half hs: query columns 64hs .. 64hs+63 of S^T / dP^T, and
+        // feature columns 64hs .. of dV / dK in the epilogue.
+        const int hs = warp / 4;
+        const int r = (warp % 4) * 32 + lane;  // TMEM lane
+        const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
         const int j = j0 + r;            // this thread's key
         // depth mode: is depth row j (slot j % Ld of token j / Ld) selected?
         const bool j_selected = !p.depth_mode || !p.depth_sel || j >= p.T * p.Ld ||
@@ -286,10 +296,12 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
         const float sl2 = p.sl2;
         const int gshift = p.gshift;
         bool ok = true;
-        // lse (log2 units) and D of row r of query tile i, loaded one tile
-        // ahead so the global-memory latency stays off the critical path.
+        // lse (log2 units) and D of query row 64hs + r (r < 64) of query tile
+        // i, loaded one tile ahead so the global-memory latency stays off the
+        // critical path.
         auto load_stat = [&](int i, float& l2, float& dd) {
-            const int t = t_first + i * n + (r >> gshift), h = kvh * p.G + (r & (p.G - 1));
+            const int rr = 64 * hs + r;
+            const int t = t_first + i * n + (rr >> gshift), h = kvh * p.G + (rr & (p.G - 1));
             if (t < p.T) {
                 const long long ix = ((long long)b * p.Hq + h) * p.T + t;
                 l2 = p.lse[ix] * kLog2e;
@@ -299,18 +311,20 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
                 dd = 0.f;
             }
         };
-        float nl2, nD;
-        load_stat(0, nl2, nD);
+        float nl2 = INFINITY, nD = 0.f;
+        if (r < 64) load_stat(0, nl2, nD);
         for (int i = 0; i < nq; ++i) {
             const int tq0 = t_first + i * n;
             float* st_lse = sStat;
             float* st_D = sStat + 128;
-            named_sync_compute();  // the previous tile's readers are done
-            st_lse[r] = nl2;
-            st_D[r] = nD;
-            if (i + 1 < nq) load_stat(i + 1, nl2, nD);
+            half_sync(hs);  // this half's readers of the previous tile are done
+            if (r < 64) {
+                st_lse[64 * hs + r] = nl2;
+                st_D[64 * hs + r] = nD;
+                if (i + 1 < nq) load_stat(i + 1, nl2, nD);
+            }
             const bool got = ptx::mbar_wait(&bars->s_full, i & 1, p.wait_limit, abort_flag);
-            if (!all_compute(got)) {  // also publishes st_lse / st_D
+            if (!half_all(hs, got)) {  // also publishes this half's st_lse / st_D
                 flag_timeout(p.status, bars);
                 ok = false;
                 break;
@@ -329,16 +343,17 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
                 hi_r = 128;
             }
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
+                const int col = 64 * hs + 32 * c;  // first query column of the chunk
                 uint32_t sr[32], dr[32];
-                ptx::tmem_ld32(tmem + lane_off + 0 + 32 * c, sr);
-                ptx::tmem_ld32(tmem + lane_off + 128 + 32 * c, dr);
+                ptx::tmem_ld32(tmem + lane_off + 0 + col, sr);
+                ptx::tmem_ld32(tmem + lane_off + 128 + col, dr);
                 ptx::tmem_wait_ld();
                 uint32_t pp[16], dd[16];
 #pragma unroll
                 for (int e2 = 0; e2 < 16; ++e2) {
                     float pv[2], dv[2];
-                    const int r0 = 32 * c + 2 * e2;
+                    const int r0 = col + 2 * e2;
                     const float2 ex = exp2_pair(make_float2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -st_lse[r0]),
                                                             fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -st_lse[r0 + 1])),
                                                 e2);
@@ -353,10 +368,10 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
                     pp[e2] = ptx::pack_bf16x2(pv[0], pv[1]);
                     dd[e2] = ptx::pack_bf16x2(dv[0], dv[1]);
                 }
-                // chunk c's packed columns [16c, 16c+16) lie in columns this
-                // thread has already read
-                ptx::tmem_st16(tmem + lane_off + 0 + 16 * c, pp);
-                ptx::tmem_st16(tmem + lane_off + 128 + 16 * c, dd);
+                // chunk c's packed columns [64hs + 16c, +16) lie in this
+                // half's columns that this thread has already read
+                ptx::tmem_st16(tmem + lane_off + 0 + 64 * hs + 16 * c, pp);
+                ptx::tmem_st16(tmem + lane_off + 128 + 64 * hs + 16 * c, dd);
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
@@ -364,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
         }
         if (ok) {
             const bool got = ptx::mbar_wait(&bars->fin, 0, p.wait_limit, abort_flag);
-            if (!all_compute(got)) {
+            if (!half_all(hs, got)) {
                 flag_timeout(p.status, bars);
                 ok = false;
             }
@@ -377,10 +392,11 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
             __nv_bfloat16* dvr = static_cast<__nv_bfloat16*>(p.dvd) + off;
             __nv_bfloat16* dkr = static_cast<__nv_bfloat16*>(p.dkd) + off;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
+                const int col = 64 * hs + 32 * c;  // feature columns of the chunk
                 uint32_t a[32], g[32];
-                ptx::tmem_ld32(tmem + lane_off + 256 + 32 * c, a);
-                ptx::tmem_ld32(tmem + lane_off + 384 + 32 * c, g);
+                ptx::tmem_ld32(tmem + lane_off + 256 + col, a);
+                ptx::tmem_ld32(tmem + lane_off + 384 + col, g);
                 ptx::tmem_wait_ld();
                 uint32_t wa[16], wg[16];
 #pragma unroll
@@ -389,8 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
                     wg[e] = ptx::pack_bf16x2(__uint_as_float(g[2 * e]) * p.scale, __uint_as_float(g[2 * e + 1]) * p.scale);
                 }
                 if (valid) {
-                    uint4* da = reinterpret_cast<uint4*>(dvr + 32 * c);
-                    uint4* dg = reinterpret_cast<uint4*>(dkr + 32 * c);
+                    uint4* da = reinterpret_cast<uint4*>(dvr + col);
+                    uint4* dg = reinterpret_cast<uint4*>(dkr + col);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         da[v] = make_uint4(wa[4 * v], wa[4 * v + 1], wa[4 * v + 2], wa[4 * v + 3]);
@@ -404,18 +420,19 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
             const bool valid = j < p.T;
             const long long off = (((long long)b * p.T + (valid ? j : 0)) * p.Hkv + kvh) * kD;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
+                const int col = 64 * hs + 32 * c;  // feature columns of the chunk
                 uint32_t a[32], g[32];
-                ptx::tmem_ld32(tmem + lane_off + 256 + 32 * c, a);
-                ptx::tmem_ld32(tmem + lane_off + 384 + 32 * c, g);
+                ptx::tmem_ld32(tmem + lane_off + 256 + col, a);
+                ptx::tmem_ld32(tmem + lane_off + 384 + col, g);
                 ptx::tmem_wait_ld();
                 if (valid) {
 #pragma unroll
                     for (int v = 0; v < 8; ++v) {
-                        red_add_v4(p.dv_acc + off + 32 * c + 4 * v, __uint_as_float(a[4 * v]),
+                        red_add_v4(p.dv_acc + off + col + 4 * v, __uint_as_float(a[4 * v]),
                                    __uint_as_float(a[4 * v + 1]), __uint_as_float(a[4 * v + 2]),
                                    __uint_as_float(a[4 * v + 3]));
-                        red_add_v4(p.dk_acc + off + 32 * c + 4 * v, __uint_as_float(g[4 * v]) * p.scale,
+                        red_add_v4(p.dk_acc + off + col + 4 * v, __uint_as_float(g[4 * v]) * p.scale,
                                    __uint_as_float(g[4 * v + 1]) * p.scale, __uint_as_float(g[4 * v + 2]) * p.scale,
                                    __uint_as_float(g[4 * v + 3]) * p.scale);
                     }
@@ -584,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
             const uint64_t km = mndesc(aRing + (sk % kDqStages) * kTile);
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k)
-                ptx::mma_ts_lead(tmem + 256, tmem + (x & 1) * 128 + k * 8, km + mnoff(k), idesc_ts,
+                ptx::mma_ts_lead(tmem + 256, tmem + (x & 1) * 128 + acol(k), km + mnoff(k), idesc_ts,
                                  (x > 0 || k > 0) ? 1u : 0u, lead);
             // K(x), V(x) are no longer needed
             ptx::mma_commit_lead(&bars->empty[sk % kDqStages], lead);
@@ -602,8 +619,11 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
         __syncwarp();
     } else {
         // ------------------------------------------------------ compute warps
-        const int r = warp * 32 + lane;  // TMEM lane = query row (token-major)
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // Column half hs: key columns 64hs .. 64hs+63 of S / dP, and feature
+        // columns 64hs .. of dQ in the epilogue.
+        const int hs = warp / 4;
+        const int r = (warp % 4) * 32 + lane;  // TMEM lane = query row (token-major)
+        const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
         const int tt = r / p.G;          // token within the tile
         const int t = t0 + tt, h = kvh * p.G + r % p.G;
         const bool row_ok = t < p.T;
@@ -627,24 +647,26 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
                 break;
             }
             ptx::tc_fence_after();
-            float pr[128];
+            float pr[64];  // P of this half's 64 key columns
             {
-                uint32_t su[128];
+                uint32_t su[64];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) ptx::tmem_ld32(rS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&su[c * 32]));
+                for (int c = 0; c < 2; ++c)
+                    ptx::tmem_ld32(rS + 64 * hs + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&su[c * 32]));
                 ptx::tmem_wait_ld();
                 uint32_t vis[4];  // visible columns of this row
                 if (x < n_kv)
                     depth_col_mask(0, t - x * kBK + 1, false, 0ull, vis);  // keys <= t
                 else  // the row's own depth rows (selected slots)
                     depth_col_mask(tt * p.Ld - (x - n_kv) * kBK, p.Ld, has_sel, sel, vis);
+                const uint32_t vw[2] = {hs ? vis[2] : vis[0], hs ? vis[3] : vis[1]};
 #pragma unroll
-                for (int c = 0; c < 128; c += 2) {
+                for (int c = 0; c < 64; c += 2) {
                     const float2 e = exp2_pair(make_float2(fmaf(__uint_as_float(su[c]), sl2, -lse2),
                                                            fmaf(__uint_as_float(su[c + 1]), sl2, -lse2)),
                                                c / 2);
-                    pr[c] = ((vis[c >> 5] >> (c & 31)) & 1u) ? e.x : 0.f;
-                    pr[c + 1] = ((vis[c >> 5] >> ((c + 1) & 31)) & 1u) ? e.y : 0.f;
+                    pr[c] = ((vw[c >> 5] >> (c & 31)) & 1u) ? e.x : 0.f;
+                    pr[c + 1] = ((vw[c >> 5] >> ((c + 1) & 31)) & 1u) ? e.y : 0.f;
                 }
             }
             if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->dp_full, x & 1, p.wait_limit, abort_flag))) {
@@ -654,9 +676,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
             }
             ptx::tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t dr[32];
-                ptx::tmem_ld32(rP + 32 * c, dr);
+                ptx::tmem_ld32(rP + 64 * hs + 32 * c, dr);
                 ptx::tmem_wait_ld();
                 uint32_t dd[16];
 #pragma unroll
@@ -665,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
                     const float d1 = pr[32 * c + 2 * e + 1] * (__uint_as_float(dr[2 * e + 1]) - Drow);
                     dd[e] = ptx::pack_bf16x2(d0, d1);
                 }
-                ptx::tmem_st16(rS + 16 * c, dd);  // over S(x), already read
+                ptx::tmem_st16(rS + 64 * hs + 16 * c, dd);  // over this half's S(x), already read
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
@@ -679,16 +701,17 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
         if (ok) {
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.dq) + (((long long)b * p.T + (row_ok ? t : 0)) * p.Hq + h) * kD;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
+                const int col = 64 * hs + 32 * c;  // feature columns of the chunk
                 uint32_t o[32];
-                ptx::tmem_ld32(tmem + lane_off + 256 + 32 * c, o);
+                ptx::tmem_ld32(tmem + lane_off + 256 + col, o);
                 ptx::tmem_wait_ld();
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
                     w[e] = ptx::pack_bf16x2(__uint_as_float(o[2 * e]) * p.scale, __uint_as_float(o[2 * e + 1]) * p.scale);
                 if (row_ok) {
-                    uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+                    uint4* d4 = reinterpret_cast<uint4*>(dst + col);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
                 }
