@@ -140,10 +140,13 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
     const int n_items = n_seq + n_dep;
     // Tile i takes part in sequence items up to its last token's tile, and in
     // the depth chunks that overlap its own tokens' depth rows.
+    // (selects rather than indexing, so that a runtime tile index keeps the
+    // arrays in registers)
     auto part = [&](int i, int x) {
-        if (x < n_seq) return x < n_kv[i];
+        const int nkv_i = i ? n_kv[1] : n_kv[0], nv_i = i ? nv[1] : nv[0];
+        if (x < n_seq) return x < nkv_i;
         const int lo = (x - n_seq) * kBN, row0 = i * n * p.Ld;
-        return nv[i] > 0 && lo < row0 + nv[i] * p.Ld && lo + kBN > row0;
+        return nv_i > 0 && lo < row0 + nv_i * p.Ld && lo + kBN > row0;
     };
 
     if (threadIdx.x == 0) {
@@ -226,12 +229,15 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
             ptx::mbar_wait(&bars->full[s % kStages], (s / kStages) & 1, kNoPollLimit, nullptr);
         __syncwarp();
     } else if (warp == kMmaWarp) {
-        // The whole warp runs the schedule so that descriptors stay
-        // warp-uniform; lane 0 issues every MMA and commit. Descriptors are
-        // formed once per tile; a K step only adds a constant to the 14-bit
-        // address field (K-major: 32 B per 16 columns within a 128-byte row,
-        // 16 KB per 64-column half; MN-major: 16 rows of 128 B = 2048 B).
-        const uint32_t lead = lane == 0;
+      // One thread runs the MMA schedule: a tcgen05.mma issued by a single
+      // thread costs about 45 cycles, against about 80 when the whole warp
+      // executes it predicated on one lane (measured on the B200), and the
+      // tensor core finishes a 128x128x16 MMA in 64 cycles, so only the
+      // single-thread form keeps it fed. Descriptors are formed once per
+      // tile; a K step only adds a constant to the 14-bit address field
+      // (K-major: 32 B per 16 columns within a 128-byte row, 16 KB per
+      // 64-column half; MN-major: 16 rows of 128 B = 2048 B).
+      if (lane == 0) {
         constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(kBM, kBN, 0, 0);
         constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, 0, 1);
         const uint32_t sQa = ptx::smem_u32(sQ);
@@ -239,10 +245,10 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
         uint64_t dq_desc[2];
         for (int i = 0; i < 2; ++i) dq_desc[i] = ptx::umma_desc_sw128(sQa + i * kTileBytes, 16, 1024);
         auto wait_all = [&](uint64_t* bar, uint32_t parity) {
-            return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, wait_limit, abort_flag));
+            return ptx::mbar_wait(bar, parity, wait_limit, abort_flag);
         };
         bool ok = wait_all(&bars->q_full, 0);
-        if (!ok && lead) flag_timeout(p, bars);
+        if (!ok) flag_timeout(p, bars);
         ptx::tc_fence_after();
         int cnt_p0 = 0, cnt_p1 = 0;
         // S_i = Q_i K^T for the K tile in ring slot `seq`
@@ -252,24 +258,24 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
         const uint64_t qd_ = dq_desc[I];                                                       \
         _Pragma("unroll") for (int k = 0; k < kD / 16; ++k) {                                  \
             const uint64_t off = (uint64_t)((k >> 2) * (kHalfBytes >> 4) + (k & 3) * 2);        \
-            ptx::mma_ss_lead(tmem + (I) * 128, qd_ + off, kd_ + off, idesc_qk, k > 0, lead);   \
+            ptx::mma_ss(tmem + (I) * 128, qd_ + off, kd_ + off, idesc_qk, k > 0);   \
         }                                                                                      \
-        ptx::mma_commit_lead(&bars->s_full[I], lead);                                          \
+        ptx::mma_commit(&bars->s_full[I]);                                          \
     } while (0)
         if (ok) ok = wait_all(&bars->full[0], 0);
-        if (!ok && lead) flag_timeout(p, bars);
+        if (!ok) flag_timeout(p, bars);
         ptx::tc_fence_after();
         if (ok) {
             if (part(0, 0)) MODA_ISSUE_S(0, 0);
             if (part(1, 0)) MODA_ISSUE_S(1, 0);
-            ptx::mma_commit_lead(&bars->empty[0], lead);
+            ptx::mma_commit(&bars->empty[0]);
         }
         for (int x = 0; x < n_items && ok; ++x) {
             const int sv = 2 * x + 1, sk = 2 * x + 2;
             const bool next = x + 1 < n_items;
             ok = wait_all(&bars->full[sv % kStages], (sv / kStages) & 1);
             if (!ok) {
-                if (lead) flag_timeout(p, bars);
+                flag_timeout(p, bars);
                 break;
             }
             ptx::tc_fence_after();
@@ -285,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
 #pragma unroll
                     for (int c = 0; c < kPChunks; ++c) {
                         if (!wait_all(&bars->p_full[i][c], cnt & 1)) {
-                            if (lead) flag_timeout(p, bars);
+                            flag_timeout(p, bars);
                             ok = false;
                             break;
                         }
@@ -293,8 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
 #pragma unroll
                         for (int kk = 0; kk < 8 / kPChunks; ++kk) {
                             const int k = (8 / kPChunks) * c + kk;
-                            ptx::mma_ts_lead(tmem + 256 + i * 128, tmem + i * 128 + k * 8, vd + (uint64_t)(k * 128),
-                                             idesc_pv, (cnt > 0 || k > 0) ? 1u : 0u, lead);
+                            ptx::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8, vd + (uint64_t)(k * 128),
+                                             idesc_pv, (cnt > 0 || k > 0) ? 1u : 0u);
                         }
                     }
                     if (!ok) break;
@@ -303,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                 if (next && part(i, x + 1)) {
                     if (!k_ready) {
                         if (!wait_all(&bars->full[sk % kStages], (sk / kStages) & 1)) {
-                            if (lead) flag_timeout(p, bars);
+                            flag_timeout(p, bars);
                             ok = false;
                             break;
                         }
@@ -314,18 +320,19 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                 }
             }
             if (!ok) break;
-            ptx::mma_commit_lead(&bars->empty[sv % kStages], lead);
-            if (next) ptx::mma_commit_lead(&bars->empty[sk % kStages], lead);
+            ptx::mma_commit(&bars->empty[sv % kStages]);
+            if (next) ptx::mma_commit(&bars->empty[sk % kStages]);
         }
 #undef MODA_ISSUE_S
         if (ok) {
-            ptx::mma_commit_lead(&bars->o_final[0], lead);
-            ptx::mma_commit_lead(&bars->o_final[1], lead);
+            ptx::mma_commit(&bars->o_final[0]);
+            ptx::mma_commit(&bars->o_final[1]);
         }
-        // Drain: all MMAs issued by this warp complete before TMEM is freed.
-        ptx::mma_commit_lead(&bars->drain, lead);
+        // Drain: all MMAs issued by this thread complete before TMEM is freed.
+        ptx::mma_commit(&bars->drain);
         ptx::mbar_wait(&bars->drain, 0, kNoPollLimit, nullptr);
-        __syncwarp();
+      }
+      __syncwarp();
     } else if (warp < 8) {
         // ------------------------------------------------ softmax warpgroups
         ptx::setmaxnreg_inc<kSoftmaxRegs>();
