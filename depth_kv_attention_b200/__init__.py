@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "MODA_OK", "ModaError", "lib", "LIB_PATH", "moda_abi_version", "moda_status_string",
     "moda_fwd", "moda_fwd_sel", "moda_bwd", "moda_bwd_sel", "moda_bwd_workspace_bytes", "moda_bwd_noalloc", "moda_pack_depth",
-    "moda_pack_depth_bytes", "moda_fwd_packed", "moda_device_status",
+    "moda_pack_depth_bytes", "moda_fwd_packed", "moda_depth_write", "moda_device_status",
     "moda_debug_set_wait_limit", "moda_debug_exp2_poly", "moda_fwd_from_host",
 ]
 
@@ -57,6 +57,7 @@ _c_bwd_sel = _sig("moda_bwd_sel", _i, [_vp] * 9 + _DIMS + [_i, _f] + [_vp] * 5 +
 _c_pack_bytes = _sig("moda_pack_depth_bytes", _sz, [_i] * 5 + [_i])
 _c_pack = _sig("moda_pack_depth", _i, [_vp, _vp] + [_i] * 5 + [_i, _vp, _vp])
 _c_fwd_packed = _sig("moda_fwd_packed", _i, [_vp] * 4 + _DIMS + [_i, _f, _vp, _vp, _vp])
+_c_depth_write = _sig("moda_depth_write", _i, [_vp, _vp] + [_i] * 6 + [_i, _vp, _vp, _vp])
 _c_dev_status = _sig("moda_device_status", _i, [_vp])
 _c_wait_limit = _sig("moda_debug_set_wait_limit", _i, [ctypes.c_uint32])
 _c_exp2_poly = _sig("moda_debug_exp2_poly", _i, [_vp, _vp, _i, _vp])
@@ -275,6 +276,22 @@ def moda_fwd_packed(q, k, v, packed, Ld: int, scale: float | None = None, out=No
                              Hkv, d, Ld, _DTYPE[q.dtype], scale, _ptr(out), _ptr(lse),
                              _stream(stream)), "moda_fwd_packed")
     return out, lse
+
+
+def moda_depth_write(k, v, kd, vd, slot: int, stream=None):
+    """The write step (``moda_depth_write``): k, v [B,T,Hkv,d] into slot
+    ``slot`` of the depth cache kd, vd [B,T,Ld,Hkv,d], in place. Returns (kd, vd)."""
+    _check_tensors(k, v, kd, vd)
+    B, T, Hkv, d = k.shape
+    Ld = kd.shape[2]
+    if tuple(v.shape) != (B, T, Hkv, d) or tuple(kd.shape) != (B, T, Ld, Hkv, d) or kd.shape != vd.shape:
+        raise ValueError("moda_depth_write: k, v [B,T,Hkv,d] and kd, vd [B,T,Ld,Hkv,d] expected")
+    if not (k.dtype == v.dtype == kd.dtype == vd.dtype):
+        raise ValueError("moda_depth_write: one dtype expected")
+    with torch.cuda.device(k.device):
+        _check(_c_depth_write(_ptr(k), _ptr(v), B, T, Hkv, d, Ld, slot, _DTYPE[k.dtype], _ptr(kd),
+                              _ptr(vd), _stream(stream)), "moda_depth_write")
+    return kd, vd
 
 
 def moda_device_status(stream=None) -> int:

@@ -240,6 +240,21 @@ moda_status moda_pack_depth(const void* kd, const void* vd, int B, int T, int Hk
     return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
 }
 
+moda_status moda_depth_write(const void* k, const void* v, int B, int T, int Hkv, int d, int Ld,
+                             int slot, moda_dtype dtype, void* kd, void* vd, void* stream) {
+    if (B < 1 || T < 1 || Hkv < 1 || d < 1 || Ld < 1) return MODA_ERR_INVALID_VALUE;
+    if (slot < 0 || slot >= Ld) return MODA_ERR_INVALID_VALUE;
+    if (dtype != MODA_BF16 && dtype != MODA_F32) return MODA_ERR_INVALID_VALUE;
+    if (!k || !v || !kd || !vd) return MODA_ERR_INVALID_VALUE;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(kd) || !aligned16(vd)) return MODA_ERR_MISALIGNED;
+    const int esz = dtype == MODA_F32 ? 4 : 2;
+    if ((d * esz) % 16) return MODA_ERR_UNSUPPORTED;  // 16-byte vector copies
+    if ((long long)B * T * Ld * Hkv * d >= (1LL << 48)) return MODA_ERR_UNSUPPORTED;
+    cudaError_t e = launch_depth_write(k, v, B, T, Hkv, d, Ld, slot, dtype, kd, vd,
+                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
+}
+
 moda_status moda_fwd_packed(const void* q, const void* k, const void* v, const void* packed_depth,
                             int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dtype,
                             float scale, void* out, float* lse, void* stream) {

@@ -73,6 +73,8 @@ cudaError_t launch_bwd_rowdot(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_depth_dkv(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_pack_depth(const void* kd, const void* vd, int B, int T, int Hkv, int d,
                               int Ld, moda_dtype dt, void* packed, cudaStream_t s);
+cudaError_t launch_depth_write(const void* k, const void* v, int B, int T, int Hkv, int d, int Ld,
+                               int slot, moda_dtype dt, void* kd, void* vd, cudaStream_t s);
 
 // Tensor-core kernels for sm_100a (moda_fwd_sm100.cu, moda_bwd_sm100.cu).
 bool fwd_tc_supported(const FwdArgs& a);

@@ -501,6 +501,42 @@ cudaError_t launch_bwd_depth_dkv(const BwdArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// The write step: k / v [B,T,Hkv,d] into slot `slot` of kd / vd
+// [B,T,Ld,Hkv,d], 16-byte vectors. One (b, t) row of k is Hkv*vec vectors
+// and lands contiguously at kd[b, t, slot], so both sides stay coalesced.
+__global__ void depth_write_kernel(const uint4* k, const uint4* v, uint4* kd, uint4* vd, long long rows,
+                                   int row_vec, int Ld, int slot) {
+    const long long per = rows * row_vec;
+    for (long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x; x < 2 * per;
+         x += (long long)gridDim.x * blockDim.x) {
+        const bool is_v = x >= per;
+        const long long y = is_v ? x - per : x;
+        const long long row = y / row_vec;  // b * T + t
+        const int c = (int)(y % row_vec);
+        const long long dst = (row * Ld + slot) * row_vec + c;
+        if (is_v) vd[dst] = v[y];
+        else kd[dst] = k[y];
+    }
+}
+
+cudaError_t launch_depth_write(const void* k, const void* v, int B, int T, int Hkv, int d, int Ld,
+                               int slot, moda_dtype dt, void* kd, void* vd, cudaStream_t s) {
+    const int esz = dt == MODA_F32 ? 4 : 2;
+    const int row_vec = Hkv * (d * esz / 16);
+    const long long rows = (long long)B * T;
+    const long long total = 2 * rows * row_vec;
+    if (total == 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    long long blocks = (total + 255) / 256;
+    if (blocks > (long long)sms * 8) blocks = (long long)sms * 8;
+    depth_write_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+                                                        static_cast<uint4*>(kd), static_cast<uint4*>(vd), rows,
+                                                        row_vec, Ld, slot);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_pack_depth(const void* kd, const void* vd, int B, int T, int Hkv, int d, int Ld,
                               moda_dtype dt, void* packed, cudaStream_t s) {
     const int esz = dt == MODA_F32 ? 4 : 2;

@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define MODA_ABI_VERSION 2
+#define MODA_ABI_VERSION 3
 
 typedef enum {
     MODA_OK = 0,
@@ -242,6 +242,25 @@ size_t moda_pack_depth_bytes(int B, int T, int Hkv, int d, int Ld, moda_dtype dt
 moda_status moda_pack_depth(const void* kd, const void* vd,
                             int B, int T, int Hkv, int d, int Ld, moda_dtype dtype,
                             void* packed, void* stream);
+
+/*
+ * moda_depth_write — the method's write step ("Mixture-of-Depths Attention",
+ * gist.science German summary §2, Write-Step): after a layer has run, its
+ * key/value pairs (for an FFN layer, the pair its light projection produced)
+ * are appended to the depth stream that later layers read. This copies
+ *   kd[b, t, slot, h, :] = k[b, t, h, :]   and   vd[b, t, slot, h, :] = v[b, t, h, :]
+ * for every b, t, h, in the native depth layout that moda_fwd reads, so no
+ * repack is needed between layers; the other slots are left untouched.
+ *   k, v   [B,T,Hkv,d]      in   the layer's keys / values (input dtype)
+ *   kd, vd [B,T,Ld,Hkv,d]   in/out  the depth cache; slot `slot` is written
+ *   slot                    in   0 <= slot < Ld, else MODA_ERR_INVALID_VALUE
+ * All pointers 16-byte aligned (MODA_ERR_MISALIGNED); d * element size must
+ * be a multiple of 16 bytes (MODA_ERR_UNSUPPORTED); k / v must not overlap
+ * kd / vd. Bit-exact copy; enqueued on `stream`.
+ */
+moda_status moda_depth_write(const void* k, const void* v,
+                             int B, int T, int Hkv, int d, int Ld, int slot,
+                             moda_dtype dtype, void* kd, void* vd, void* stream);
 
 /* moda_fwd reading depth keys/values from moda_pack_depth's layout. */
 moda_status moda_fwd_packed(const void* q, const void* k, const void* v,

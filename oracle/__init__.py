@@ -4,4 +4,4 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU baseline
 and reference arm may import this package. It shares no code with the CUDA
 path and imports nothing from it.
 """
-from .moda_oracle import backward, forward, forward_rows, to_f64  # noqa: F401
+from .moda_oracle import backward, depth_write, forward, forward_rows, to_f64  # noqa: F401

@@ -54,7 +54,7 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["to_f64", "forward", "forward_rows", "backward"]
+__all__ = ["to_f64", "forward", "forward_rows", "backward", "depth_write"]
 
 
 def to_f64(x) -> np.ndarray:
@@ -214,3 +214,16 @@ def backward(q, k, v, kd, vd, dout, scale: float, row_block: int = 256, out_for_
                 dkd[b, t0:t1, :, g] += scale * dS_dep[:, :, None] * qr[:, None, :]
                 dvd[b, t0:t1, :, g] += P_dep[:, :, None] * dor[:, None, :]
     return dq, dk, dv, dkd, dvd, out, lse
+
+
+def depth_write(kd, vd, k, v, slot: int):
+    """The write step ("Mixture-of-Depths Attention", gist.science German
+    summary §2, Write-Step): the layer's keys / values k, v [B,T,Hkv,d] are
+    appended to the depth stream as slot ``slot`` of every token's depth
+    entries. Returns new arrays kd', vd' [B,T,Ld,Hkv,d] equal to kd, vd except
+    kd'[:, :, slot] = k and vd'[:, :, slot] = v (values unchanged: a copy)."""
+    kd2 = np.array(kd, copy=True)
+    vd2 = np.array(vd, copy=True)
+    kd2[:, :, slot] = np.asarray(k)
+    vd2[:, :, slot] = np.asarray(v)
+    return kd2, vd2

@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_status_strings():
-    assert moda.moda_abi_version() == 2
+    assert moda.moda_abi_version() == 3
     assert moda.moda_status_string(0) == "MODA_OK"
     assert moda.moda_status_string(6) == "MODA_ERR_DEVICE_TIMEOUT"
     assert moda.moda_status_string(99) == "MODA_ERR_UNKNOWN"
@@ -107,3 +107,18 @@ def test_selection_validation():
     assert bwd_sel(sel=P + 4) == 3
     assert bwd_sel(Ld=65) == 2
     assert bwd_sel(dq=None) == 1
+
+
+def depth_write(slot=1, Ld=3, d=64, dt=0, k=P, kd=P):
+    return moda._c_depth_write(k, P, 2, 5, 2, d, Ld, slot, dt, kd, P, None)
+
+
+def test_depth_write_validation():
+    """The write step rejects a slot outside [0, Ld), NULL or misaligned
+    buffers, and rows that are not whole 16-byte vectors."""
+    assert depth_write(slot=3) == 1
+    assert depth_write(slot=-1) == 1
+    assert depth_write(Ld=0, slot=0) == 1
+    assert depth_write(k=None) == 1
+    assert depth_write(kd=P + 8) == 3
+    assert depth_write(d=12) == 2          # 24 bytes per bf16 row

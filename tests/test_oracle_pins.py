@@ -421,3 +421,42 @@ def test_planted_selection_mistakes_are_caught(monkeypatch):
         monkeypatch.setattr(om, "_sel", fn)
         assert not sel_pins_pass(), name
         monkeypatch.setattr(om, "_sel", orig_sel)
+
+
+# ---------------------------------------------------------------- write step
+def test_depth_write_against_loops_and_forward():
+    """The write step against scalar loops (only slot `slot` of every token
+    changes), and a depth cache filled layer by layer equals one whose depth
+    axis holds the layers' keys / values in order, as the forward reads it."""
+    rng = np.random.default_rng(41)
+    B, T, Ld, Hkv, d = 2, 5, 3, 2, 4
+    kd = rng.standard_normal((B, T, Ld, Hkv, d))
+    vd = rng.standard_normal((B, T, Ld, Hkv, d))
+    k = rng.standard_normal((B, T, Hkv, d))
+    v = rng.standard_normal((B, T, Hkv, d))
+    kd_before = kd.copy()
+    kd2, vd2 = om.depth_write(kd, vd, k, v, 1)
+    for b in range(B):
+        for t in range(T):
+            for i in range(Ld):
+                for h in range(Hkv):
+                    for c in range(d):
+                        ek = k[b, t, h, c] if i == 1 else kd[b, t, i, h, c]
+                        ev = v[b, t, h, c] if i == 1 else vd[b, t, i, h, c]
+                        assert kd2[b, t, i, h, c] == ek and vd2[b, t, i, h, c] == ev
+    assert np.array_equal(kd, kd_before)  # the inputs are not modified
+    # layer by layer into an empty cache, then the forward of the next layer
+    Hq = 4
+    layers = [(rng.standard_normal((B, T, Hkv, d)), rng.standard_normal((B, T, Hkv, d))) for _ in range(Ld)]
+    ckd = np.zeros((B, T, Ld, Hkv, d))
+    cvd = np.zeros((B, T, Ld, Hkv, d))
+    for slot, (kl, vl) in enumerate(layers):
+        ckd, cvd = om.depth_write(ckd, cvd, kl, vl, slot)
+    q = rng.standard_normal((B, T, Hq, d))
+    ks, vs = rng.standard_normal((B, T, Hkv, d)), rng.standard_normal((B, T, Hkv, d))
+    o1, l1 = om.forward(q, ks, vs, ckd, cvd, 0.5)
+    stacked_k = np.stack([kl for kl, _ in layers], axis=2)
+    stacked_v = np.stack([vl for _, vl in layers], axis=2)
+    o2, l2 = brute_force(q, ks, vs, stacked_k, stacked_v, 0.5)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-12)
