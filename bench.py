@@ -16,6 +16,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -312,16 +313,26 @@ def measure_secondary(moda, w, world, kernel, steps=5, warmup=3):
     return res
 
 
+def code_hash(path: str) -> str:
+    """SHA-256 (16 hex digits) of a CUDA source with its comments and all
+    whitespace removed: it changes when the code changes, not when a comment
+    or the layout does."""
+    with open(path) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    src = re.sub(r"\s+", "", src)
+    return hashlib.sha256(src.encode()).hexdigest()[:16]
+
+
 def traffic_for(kernel_src: str):
     """DRAM bytes per launch from the committed ncu summary, or None when the
-    kernel source changed since the counters were taken."""
+    kernel's code changed since the counters were taken."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         t = json.load(f)
-    with open(kernel_src, "rb") as f:
-        h = hashlib.sha256(f.read()).hexdigest()[:16]
-    if t.get("source_sha256_16") != h:
+    if t.get("code_sha256_16") != code_hash(kernel_src):
         return None
     return t.get("dram_bytes_per_launch")
 

@@ -244,51 +244,51 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
             ptx::mbar_wait(&bars->full[i % kDkvStages], (i / kDkvStages) & 1, 0, nullptr);
         __syncwarp();
     } else if (warp == kMmaWarp) {
-      // One thread runs the MMA schedule (a single-thread tcgen05.mma issue
-      // costs about 45 cycles, a warp-wide one predicated on one lane about
-      // 80, against 64 cycles of tensor work for a 128x128x16 MMA).
-      if (lane == 0) {
-        constexpr uint32_t idesc_ss = ptx::idesc_bf16_f32(128, 128, 0, 0);
-        constexpr uint32_t idesc_ts = ptx::idesc_bf16_f32(128, kD, 0, 1);
-        const uint64_t dK = kdesc(ptx::smem_u32(sK)), dV = kdesc(ptx::smem_u32(sV));
-        const uint32_t aRing = ptx::smem_u32(sRing);
-        bool ok = wait_one(&bars->kv_full, 0);
-        if (!ok) flag_timeout(p.status, bars);
-        ptx::tc_fence_after();
-        for (int i = 0; i < nq && ok; ++i) {
-            const int st = i % kDkvStages;
-            const uint32_t aQ = aRing + (2 * st) * kTile, aDO = aRing + (2 * st + 1) * kTile;
-            ok = wait_one(&bars->full[st], (i / kDkvStages) & 1);
-            if (!ok) {
-                flag_timeout(p.status, bars);
-                break;
-            }
+        // One thread runs the MMA schedule (a single-thread tcgen05.mma issue
+        // costs about 45 cycles, a warp-wide one predicated on one lane about
+        // 80, against 64 cycles of tensor work for a 128x128x16 MMA).
+        if (lane == 0) {
+            constexpr uint32_t idesc_ss = ptx::idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t idesc_ts = ptx::idesc_bf16_f32(128, kD, 0, 1);
+            const uint64_t dK = kdesc(ptx::smem_u32(sK)), dV = kdesc(ptx::smem_u32(sV));
+            const uint32_t aRing = ptx::smem_u32(sRing);
+            bool ok = wait_one(&bars->kv_full, 0);
+            if (!ok) flag_timeout(p.status, bars);
             ptx::tc_fence_after();
-            const uint64_t dQk = kdesc(aQ), dOk = kdesc(aDO), dQm = mndesc(aQ), dOm = mndesc(aDO);
+            for (int i = 0; i < nq && ok; ++i) {
+                const int st = i % kDkvStages;
+                const uint32_t aQ = aRing + (2 * st) * kTile, aDO = aRing + (2 * st + 1) * kTile;
+                ok = wait_one(&bars->full[st], (i / kDkvStages) & 1);
+                if (!ok) {
+                    flag_timeout(p.status, bars);
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint64_t dQk = kdesc(aQ), dOk = kdesc(aDO), dQm = mndesc(aQ), dOm = mndesc(aDO);
 #pragma unroll
-            for (int k = 0; k < kD / 16; ++k) ptx::mma_ss(tmem + 0, dK + koff(k), dQk + koff(k), idesc_ss, k > 0);
+                for (int k = 0; k < kD / 16; ++k) ptx::mma_ss(tmem + 0, dK + koff(k), dQk + koff(k), idesc_ss, k > 0);
 #pragma unroll
-            for (int k = 0; k < kD / 16; ++k) ptx::mma_ss(tmem + 128, dV + koff(k), dOk + koff(k), idesc_ss, k > 0);
-            ptx::mma_commit(&bars->s_full);
-            if (!wait_one(&bars->p_full, i & 1)) {
-                flag_timeout(p.status, bars);
-                ok = false;
-                break;
+                for (int k = 0; k < kD / 16; ++k) ptx::mma_ss(tmem + 128, dV + koff(k), dOk + koff(k), idesc_ss, k > 0);
+                ptx::mma_commit(&bars->s_full);
+                if (!wait_one(&bars->p_full, i & 1)) {
+                    flag_timeout(p.status, bars);
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 128 / 16; ++k)
+                    ptx::mma_ts(tmem + 256, tmem + 0 + acol(k), dOm + mnoff(k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                for (int k = 0; k < 128 / 16; ++k)
+                    ptx::mma_ts(tmem + 384, tmem + 128 + acol(k), dQm + mnoff(k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u);
+                ptx::mma_commit(&bars->empty[st]);
             }
-            ptx::tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 128 / 16; ++k)
-                ptx::mma_ts(tmem + 256, tmem + 0 + acol(k), dOm + mnoff(k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-            for (int k = 0; k < 128 / 16; ++k)
-                ptx::mma_ts(tmem + 384, tmem + 128 + acol(k), dQm + mnoff(k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u);
-            ptx::mma_commit(&bars->empty[st]);
+            if (ok) ptx::mma_commit(&bars->fin);
+            ptx::mma_commit(&bars->drain);
+            ptx::mbar_wait(&bars->drain, 0, 0, nullptr);
         }
-        if (ok) ptx::mma_commit(&bars->fin);
-        ptx::mma_commit(&bars->drain);
-        ptx::mbar_wait(&bars->drain, 0, 0, nullptr);
-      }
-      __syncwarp();
+        __syncwarp();
     } else {
         // ------------------------------------------------------ compute warps
         // Column half hs: query columns 64hs .. 64hs+63 of S^T / dP^T, and
@@ -563,74 +563,74 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
             ptx::mbar_wait(&bars->full[s % kDqStages], (s / kDqStages) & 1, 0, nullptr);
         __syncwarp();
     } else if (warp == kMmaWarp) {
-      // One thread runs the MMA schedule (a single-thread tcgen05.mma issue
-      // costs about 45 cycles, a warp-wide one predicated on one lane about
-      // 80, against 64 cycles of tensor work for a 128x128x16 MMA).
-      if (lane == 0) {
-        constexpr uint32_t idesc_ss = ptx::idesc_bf16_f32(128, 128, 0, 0);
-        constexpr uint32_t idesc_ts = ptx::idesc_bf16_f32(128, kD, 0, 1);
-        const uint64_t dQk = kdesc(ptx::smem_u32(sQ)), dOk = kdesc(ptx::smem_u32(sDO));
-        const uint32_t aRing = ptx::smem_u32(sRing);
-        bool ok = wait_one(&bars->kv_full, 0);
-        if (!ok) flag_timeout(p.status, bars);
-        ptx::tc_fence_after();
-        // ring slots: item x has K at 2x, V at 2x+1
-        auto issue_s = [&](int x) {  // S(x) = Q K(x)^T into R[x % 2]
-            const int sk = 2 * x;
-            if (!wait_one(&bars->full[sk % kDqStages], (sk / kDqStages) & 1)) return false;
+        // One thread runs the MMA schedule (a single-thread tcgen05.mma issue
+        // costs about 45 cycles, a warp-wide one predicated on one lane about
+        // 80, against 64 cycles of tensor work for a 128x128x16 MMA).
+        if (lane == 0) {
+            constexpr uint32_t idesc_ss = ptx::idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t idesc_ts = ptx::idesc_bf16_f32(128, kD, 0, 1);
+            const uint64_t dQk = kdesc(ptx::smem_u32(sQ)), dOk = kdesc(ptx::smem_u32(sDO));
+            const uint32_t aRing = ptx::smem_u32(sRing);
+            bool ok = wait_one(&bars->kv_full, 0);
+            if (!ok) flag_timeout(p.status, bars);
             ptx::tc_fence_after();
-            const uint64_t kk = kdesc(aRing + (sk % kDqStages) * kTile);
+            // ring slots: item x has K at 2x, V at 2x+1
+            auto issue_s = [&](int x) {  // S(x) = Q K(x)^T into R[x % 2]
+                const int sk = 2 * x;
+                if (!wait_one(&bars->full[sk % kDqStages], (sk / kDqStages) & 1)) return false;
+                ptx::tc_fence_after();
+                const uint64_t kk = kdesc(aRing + (sk % kDqStages) * kTile);
 #pragma unroll
-            for (int k = 0; k < kD / 16; ++k)
-                ptx::mma_ss(tmem + (x & 1) * 128, dQk + koff(k), kk + koff(k), idesc_ss, k > 0);
-            ptx::mma_commit(&bars->s_full);
-            return true;
-        };
-        auto issue_dp = [&](int x) {  // dP(x) = dO V(x)^T into R[(x + 1) % 2]
-            const int sv = 2 * x + 1;
-            if (!wait_one(&bars->full[sv % kDqStages], (sv / kDqStages) & 1)) return false;
-            ptx::tc_fence_after();
-            const uint64_t vk = kdesc(aRing + (sv % kDqStages) * kTile);
+                for (int k = 0; k < kD / 16; ++k)
+                    ptx::mma_ss(tmem + (x & 1) * 128, dQk + koff(k), kk + koff(k), idesc_ss, k > 0);
+                ptx::mma_commit(&bars->s_full);
+                return true;
+            };
+            auto issue_dp = [&](int x) {  // dP(x) = dO V(x)^T into R[(x + 1) % 2]
+                const int sv = 2 * x + 1;
+                if (!wait_one(&bars->full[sv % kDqStages], (sv / kDqStages) & 1)) return false;
+                ptx::tc_fence_after();
+                const uint64_t vk = kdesc(aRing + (sv % kDqStages) * kTile);
 #pragma unroll
-            for (int k = 0; k < kD / 16; ++k)
-                ptx::mma_ss(tmem + ((x + 1) & 1) * 128, dOk + koff(k), vk + koff(k), idesc_ss, k > 0);
-            ptx::mma_commit(&bars->dp_full);
-            return true;
-        };
-        if (ok) ok = issue_s(0) && issue_dp(0);
-        for (int x = 0; x < n_items && ok; ++x) {
-            // dS(x) is in R[x % 2]; the compute warps have read dP(x) from
-            // R[(x + 1) % 2], which S(x + 1) may now overwrite.
-            if (!wait_one(&bars->p_full, x & 1)) {
-                ok = false;
-                break;
-            }
-            ptx::tc_fence_after();
-            if (x + 1 < n_items && !issue_s(x + 1)) {
-                ok = false;
-                break;
-            }
-            const int sk = 2 * x;
-            const uint64_t km = mndesc(aRing + (sk % kDqStages) * kTile);
+                for (int k = 0; k < kD / 16; ++k)
+                    ptx::mma_ss(tmem + ((x + 1) & 1) * 128, dOk + koff(k), vk + koff(k), idesc_ss, k > 0);
+                ptx::mma_commit(&bars->dp_full);
+                return true;
+            };
+            if (ok) ok = issue_s(0) && issue_dp(0);
+            for (int x = 0; x < n_items && ok; ++x) {
+                // dS(x) is in R[x % 2]; the compute warps have read dP(x) from
+                // R[(x + 1) % 2], which S(x + 1) may now overwrite.
+                if (!wait_one(&bars->p_full, x & 1)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                if (x + 1 < n_items && !issue_s(x + 1)) {
+                    ok = false;
+                    break;
+                }
+                const int sk = 2 * x;
+                const uint64_t km = mndesc(aRing + (sk % kDqStages) * kTile);
 #pragma unroll
-            for (int k = 0; k < kBK / 16; ++k)
-                ptx::mma_ts(tmem + 256, tmem + (x & 1) * 128 + acol(k), km + mnoff(k), idesc_ts,
-                                 (x > 0 || k > 0) ? 1u : 0u);
-            // K(x), V(x) are no longer needed
-            ptx::mma_commit(&bars->empty[sk % kDqStages]);
-            ptx::mma_commit(&bars->empty[(sk + 1) % kDqStages]);
-            // dP(x + 1) into R[x % 2], after dQ has read dS(x) there
-            if (x + 1 < n_items && !issue_dp(x + 1)) {
-                ok = false;
-                break;
+                for (int k = 0; k < kBK / 16; ++k)
+                    ptx::mma_ts(tmem + 256, tmem + (x & 1) * 128 + acol(k), km + mnoff(k), idesc_ts,
+                                     (x > 0 || k > 0) ? 1u : 0u);
+                // K(x), V(x) are no longer needed
+                ptx::mma_commit(&bars->empty[sk % kDqStages]);
+                ptx::mma_commit(&bars->empty[(sk + 1) % kDqStages]);
+                // dP(x + 1) into R[x % 2], after dQ has read dS(x) there
+                if (x + 1 < n_items && !issue_dp(x + 1)) {
+                    ok = false;
+                    break;
+                }
             }
+            if (!ok) flag_timeout(p.status, bars);
+            if (ok) ptx::mma_commit(&bars->fin);
+            ptx::mma_commit(&bars->drain);
+            ptx::mbar_wait(&bars->drain, 0, 0, nullptr);
         }
-        if (!ok) flag_timeout(p.status, bars);
-        if (ok) ptx::mma_commit(&bars->fin);
-        ptx::mma_commit(&bars->drain);
-        ptx::mbar_wait(&bars->drain, 0, 0, nullptr);
-      }
-      __syncwarp();
+        __syncwarp();
     } else {
         // ------------------------------------------------------ compute warps
         // Column half hs: key columns 64hs .. 64hs+63 of S / dP, and feature

@@ -22,8 +22,9 @@
 //    depth range is read). Each depth row is read once per unit.
 //  * Warp roles: warps 0-3 and 4-7 run the softmax of query tiles 0 and 1
 //    (one thread per row, TMEM lane = row); warp 8 issues TMA loads into a
-//    4-stage ring; warp 9 issues tcgen05.mma (warps 10-11 only pad the
-//    third warpgroup for the register reallocation). TMEM: S0 | S1 | O0 | O1, 128
+//    5-stage ring; lane 0 of warp 9 issues every tcgen05.mma (warps 10-11
+//    only pad the third warpgroup for the register reallocation).
+//    TMEM: S0 | S1 | O0 | O1, 128
 //    fp32 columns each; P (bf16) overwrites the first 64 columns of S and is
 //    the TMEM A operand of O += P V. While tile 0's softmax runs, the tensor
 //    core computes tile 1's S, and the other way round.
@@ -229,29 +230,30 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
             ptx::mbar_wait(&bars->full[s % kStages], (s / kStages) & 1, kNoPollLimit, nullptr);
         __syncwarp();
     } else if (warp == kMmaWarp) {
-      // One thread runs the MMA schedule: a tcgen05.mma issued by a single
-      // thread costs about 45 cycles, against about 80 when the whole warp
-      // executes it predicated on one lane (measured on the B200), and the
-      // tensor core finishes a 128x128x16 MMA in 64 cycles, so only the
-      // single-thread form keeps it fed. Descriptors are formed once per
-      // tile; a K step only adds a constant to the 14-bit address field
-      // (K-major: 32 B per 16 columns within a 128-byte row, 16 KB per
-      // 64-column half; MN-major: 16 rows of 128 B = 2048 B).
-      if (lane == 0) {
-        constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(kBM, kBN, 0, 0);
-        constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, 0, 1);
-        const uint32_t sQa = ptx::smem_u32(sQ);
-        const uint32_t sRa = ptx::smem_u32(sRing);
-        uint64_t dq_desc[2];
-        for (int i = 0; i < 2; ++i) dq_desc[i] = ptx::umma_desc_sw128(sQa + i * kTileBytes, 16, 1024);
-        auto wait_all = [&](uint64_t* bar, uint32_t parity) {
-            return ptx::mbar_wait(bar, parity, wait_limit, abort_flag);
-        };
-        bool ok = wait_all(&bars->q_full, 0);
-        if (!ok) flag_timeout(p, bars);
-        ptx::tc_fence_after();
-        int cnt_p0 = 0, cnt_p1 = 0;
-        // S_i = Q_i K^T for the K tile in ring slot `seq`
+        // One thread runs the MMA schedule: a tcgen05.mma issued by a single
+        // thread costs about 45 cycles, against about 80 when the whole warp
+        // executes it predicated on one lane (measured on the B200), and the
+        // tensor core finishes a 128x128x16 MMA in 64 cycles, so only the
+        // single-thread form keeps it fed. Descriptors are formed once per
+        // tile; a K step only adds a constant to the 14-bit address field
+        // (K-major: 32 B per 16 columns within a 128-byte row, 16 KB per
+        // 64-column half; MN-major: 16 rows of 128 B = 2048 B).
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(kBM, kBN, 0, 0);
+            constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBM, kD, 0, 1);
+            const uint32_t sQa = ptx::smem_u32(sQ);
+            const uint32_t sRa = ptx::smem_u32(sRing);
+            uint64_t dq_desc[2];
+            for (int i = 0; i < 2; ++i) dq_desc[i] = ptx::umma_desc_sw128(sQa + i * kTileBytes, 16, 1024);
+            // (a plain bounded wait: one thread, no warp vote)
+            auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+                return ptx::mbar_wait(bar, parity, wait_limit, abort_flag);
+            };
+            bool ok = wait_all(&bars->q_full, 0);
+            if (!ok) flag_timeout(p, bars);
+            ptx::tc_fence_after();
+            int cnt_p0 = 0, cnt_p1 = 0;
+            // S_i = Q_i K^T for the K tile in ring slot `seq`
 #define MODA_ISSUE_S(I, SEQ)                                                                   \
     do {                                                                                       \
         const uint64_t kd_ = ptx::umma_desc_sw128(sRa + ((SEQ) % kStages) * kTileBytes, 16, 1024); \
@@ -262,77 +264,77 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
         }                                                                                      \
         ptx::mma_commit(&bars->s_full[I]);                                          \
     } while (0)
-        if (ok) ok = wait_all(&bars->full[0], 0);
-        if (!ok) flag_timeout(p, bars);
-        ptx::tc_fence_after();
-        if (ok) {
-            if (part(0, 0)) MODA_ISSUE_S(0, 0);
-            if (part(1, 0)) MODA_ISSUE_S(1, 0);
-            ptx::mma_commit(&bars->empty[0]);
-        }
-        for (int x = 0; x < n_items && ok; ++x) {
-            const int sv = 2 * x + 1, sk = 2 * x + 2;
-            const bool next = x + 1 < n_items;
-            ok = wait_all(&bars->full[sv % kStages], (sv / kStages) & 1);
-            if (!ok) {
-                flag_timeout(p, bars);
-                break;
-            }
+            if (ok) ok = wait_all(&bars->full[0], 0);
+            if (!ok) flag_timeout(p, bars);
             ptx::tc_fence_after();
-            const uint64_t vd = ptx::umma_desc_sw128(sRa + (sv % kStages) * kTileBytes, kHalfBytes, 1024);
-            bool k_ready = false;
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                if (!ok) break;
-                if (part(i, x)) {
-                    // O_i += P_i V, fed chunk by chunk as the softmax
-                    // publishes P (32 keys per chunk = 2 MMA K-steps).
-                    const int cnt = i ? cnt_p1 : cnt_p0;
-#pragma unroll
-                    for (int c = 0; c < kPChunks; ++c) {
-                        if (!wait_all(&bars->p_full[i][c], cnt & 1)) {
-                            flag_timeout(p, bars);
-                            ok = false;
-                            break;
-                        }
-                        ptx::tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < 8 / kPChunks; ++kk) {
-                            const int k = (8 / kPChunks) * c + kk;
-                            ptx::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8, vd + (uint64_t)(k * 128),
-                                             idesc_pv, (cnt > 0 || k > 0) ? 1u : 0u);
-                        }
-                    }
-                    if (!ok) break;
-                    if (i) ++cnt_p1; else ++cnt_p0;
-                }
-                if (next && part(i, x + 1)) {
-                    if (!k_ready) {
-                        if (!wait_all(&bars->full[sk % kStages], (sk / kStages) & 1)) {
-                            flag_timeout(p, bars);
-                            ok = false;
-                            break;
-                        }
-                        ptx::tc_fence_after();
-                        k_ready = true;
-                    }
-                    MODA_ISSUE_S(i, sk);
-                }
+            if (ok) {
+                if (part(0, 0)) MODA_ISSUE_S(0, 0);
+                if (part(1, 0)) MODA_ISSUE_S(1, 0);
+                ptx::mma_commit(&bars->empty[0]);
             }
-            if (!ok) break;
-            ptx::mma_commit(&bars->empty[sv % kStages]);
-            if (next) ptx::mma_commit(&bars->empty[sk % kStages]);
-        }
+            for (int x = 0; x < n_items && ok; ++x) {
+                const int sv = 2 * x + 1, sk = 2 * x + 2;
+                const bool next = x + 1 < n_items;
+                ok = wait_all(&bars->full[sv % kStages], (sv / kStages) & 1);
+                if (!ok) {
+                    flag_timeout(p, bars);
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint64_t vd = ptx::umma_desc_sw128(sRa + (sv % kStages) * kTileBytes, kHalfBytes, 1024);
+                bool k_ready = false;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    if (!ok) break;
+                    if (part(i, x)) {
+                        // O_i += P_i V, fed chunk by chunk as the softmax
+                        // publishes P (32 keys per chunk = 2 MMA K-steps).
+                        const int cnt = i ? cnt_p1 : cnt_p0;
+#pragma unroll
+                        for (int c = 0; c < kPChunks; ++c) {
+                            if (!wait_all(&bars->p_full[i][c], cnt & 1)) {
+                                flag_timeout(p, bars);
+                                ok = false;
+                                break;
+                            }
+                            ptx::tc_fence_after();
+#pragma unroll
+                            for (int kk = 0; kk < 8 / kPChunks; ++kk) {
+                                const int k = (8 / kPChunks) * c + kk;
+                                ptx::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8, vd + (uint64_t)(k * 128),
+                                                 idesc_pv, (cnt > 0 || k > 0) ? 1u : 0u);
+                            }
+                        }
+                        if (!ok) break;
+                        if (i) ++cnt_p1; else ++cnt_p0;
+                    }
+                    if (next && part(i, x + 1)) {
+                        if (!k_ready) {
+                            if (!wait_all(&bars->full[sk % kStages], (sk / kStages) & 1)) {
+                                flag_timeout(p, bars);
+                                ok = false;
+                                break;
+                            }
+                            ptx::tc_fence_after();
+                            k_ready = true;
+                        }
+                        MODA_ISSUE_S(i, sk);
+                    }
+                }
+                if (!ok) break;
+                ptx::mma_commit(&bars->empty[sv % kStages]);
+                if (next) ptx::mma_commit(&bars->empty[sk % kStages]);
+            }
 #undef MODA_ISSUE_S
-        if (ok) {
-            ptx::mma_commit(&bars->o_final[0]);
-            ptx::mma_commit(&bars->o_final[1]);
+            if (ok) {
+                ptx::mma_commit(&bars->o_final[0]);
+                ptx::mma_commit(&bars->o_final[1]);
+            }
+            // Drain: all MMAs issued by this thread complete before TMEM is freed.
+            ptx::mma_commit(&bars->drain);
+            ptx::mbar_wait(&bars->drain, 0, kNoPollLimit, nullptr);
         }
-        // Drain: all MMAs issued by this thread complete before TMEM is freed.
-        ptx::mma_commit(&bars->drain);
-        ptx::mbar_wait(&bars->drain, 0, kNoPollLimit, nullptr);
-      }
-      __syncwarp();
+        __syncwarp();
     } else if (warp < 8) {
         // ------------------------------------------------ softmax warpgroups
         ptx::setmaxnreg_inc<kSoftmaxRegs>();
