@@ -101,7 +101,7 @@ struct __align__(8) Bars {
     uint64_t kv_full;            // dk/dv kernel: K, V tile | dq kernel: Q, dO tile
     uint64_t full[4];            // ring slots
     uint64_t empty[4];
-    uint64_t s_full, dp_full, p_full, fin, drain;
+    uint64_t s_full, dp_full, p_full, p_full2, fin, drain;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -111,7 +111,10 @@ __device__ __forceinline__ void flag_timeout(unsigned int* status, Bars* bars) {
     atomicOr(status, 1u);
 }
 
-__device__ __forceinline__ void init_bars(Bars* bars, int stages) {
+// p_count: arrivals that publish P (the dQ kernel: all 256 compute threads
+// on p_full; the dK/dV kernel: each 128-thread half on its own p_full /
+// p_full2).
+__device__ __forceinline__ void init_bars(Bars* bars, int stages, int p_count) {
     ptx::mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < stages; ++s) {
         ptx::mbar_init(&bars->full[s], 1);
@@ -119,7 +122,8 @@ __device__ __forceinline__ void init_bars(Bars* bars, int stages) {
     }
     ptx::mbar_init(&bars->s_full, 1);
     ptx::mbar_init(&bars->dp_full, 1);
-    ptx::mbar_init(&bars->p_full, kComputeThreads);
+    ptx::mbar_init(&bars->p_full, p_count);
+    ptx::mbar_init(&bars->p_full2, p_count);
     ptx::mbar_init(&bars->fin, 1);
     ptx::mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -156,12 +160,17 @@ static_assert(sizeof(Bars) <= 256, "barrier block");
 // tiles are those holding the chunk's tokens, the mask keeps each depth row
 // to its own token's G heads, and since one CTA owns every row of its chunk
 // the results are written directly in bf16.
-// TMEM: S^T | dP^T | dV | dK, 128 columns each.
-// Per query tile: S^T = K Q^T, dP^T = V dO^T; the compute warps (thread =
-// key) form P^T and dS^T in bf16 over S^T / dP^T; dV += P^T dO and
-// dK += dS^T Q take them as TMEM A operands. The next tile's S^T / dP^T
-// follow those two MMAs in issue order, so they overwrite P^T / dS^T only
-// after they are read.
+// Each 128-row query tile is processed as two halves of 64 query rows that
+// ping-pong like the forward's two query tiles: while the compute warps of
+// one half form P^T and dS^T, the tensor core runs the other half's MMAs.
+// TMEM: [S^T | dP^T] of half 0, [S^T | dP^T] of half 1 (64 columns each),
+// then dV | dK (128 columns each).
+// Per half h of query tile i: S^T_h = K Q_h^T and dP^T_h = V dO_h^T
+// (N = 64); the 128 compute threads of half h (thread = key) write P^T_h and
+// dS^T_h in bf16 over them; dV += P^T_h dO_h and dK += dS^T_h Q_h take them
+// as TMEM A operands (K = 64 queries). MMA issue order per tile:
+// PV_0(i), S/dP_0(i+1), PV_1(i), S/dP_1(i+1), so a half's next S^T / dP^T
+// overwrite its P^T / dS^T only after they are read.
 __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid_constant__ DkvParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -193,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
         nq = (c_hi - t_first + n - 1) / n;
     }
 
-    if (threadIdx.x == 0) init_bars(bars, kDkvStages);
+    if (threadIdx.x == 0) init_bars(bars, kDkvStages, kComputeThreads / 2);
     if (warp == 0) {
         ptx::tmem_alloc(&bars->tmem_base, 512);
         ptx::tmem_relinquish();
@@ -248,41 +257,72 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
         // costs about 45 cycles, a warp-wide one predicated on one lane about
         // 80, against 64 cycles of tensor work for a 128x128x16 MMA).
         if (lane == 0) {
-            constexpr uint32_t idesc_ss = ptx::idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t idesc_half = ptx::idesc_bf16_f32(128, 64, 0, 0);
             constexpr uint32_t idesc_ts = ptx::idesc_bf16_f32(128, kD, 0, 1);
             const uint64_t dK = kdesc(ptx::smem_u32(sK)), dV = kdesc(ptx::smem_u32(sV));
             const uint32_t aRing = ptx::smem_u32(sRing);
-            bool ok = wait_one(&bars->kv_full, 0);
+            uint64_t* s_ready[2] = {&bars->s_full, &bars->dp_full};
+            uint64_t* p_ready[2] = {&bars->p_full, &bars->p_full2};
+            // S^T_h = K Q_h^T and dP^T_h = V dO_h^T for query half h of the
+            // tile in ring stage st (rows 64h.. of each 64-column half of the
+            // K-major Q / dO tile: 64 rows of 128 B = 512 descriptor units)
+            auto issue_sdp = [&](int st, int h) {
+                const uint32_t aQ = aRing + (2 * st) * kTile, aDO = aRing + (2 * st + 1) * kTile;
+                const uint64_t rows = (uint64_t)(h * 512);
+                const uint64_t dQk = kdesc(aQ) + rows, dOk = kdesc(aDO) + rows;
+#pragma unroll
+                for (int k = 0; k < kD / 16; ++k)
+                    ptx::mma_ss(tmem + 128 * h, dK + koff(k), dQk + koff(k), idesc_half, k > 0);
+#pragma unroll
+                for (int k = 0; k < kD / 16; ++k)
+                    ptx::mma_ss(tmem + 128 * h + 64, dV + koff(k), dOk + koff(k), idesc_half, k > 0);
+                ptx::mma_commit(s_ready[h]);
+            };
+            // dV += P^T_h dO_h and dK += dS^T_h Q_h: K steps 4h .. 4h+3 of the
+            // MN-major dO / Q tile, A operands from half h's TMEM columns
+            auto issue_pv = [&](int st, int h, bool first) {
+                const uint32_t aQ = aRing + (2 * st) * kTile, aDO = aRing + (2 * st + 1) * kTile;
+                const uint64_t dQm = mndesc(aQ), dOm = mndesc(aDO);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    ptx::mma_ts(tmem + 256, tmem + 128 * h + 8 * kk, dOm + mnoff(4 * h + kk), idesc_ts,
+                                (first && kk == 0) ? 0u : 1u);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    ptx::mma_ts(tmem + 384, tmem + 128 * h + 64 + 8 * kk, dQm + mnoff(4 * h + kk), idesc_ts,
+                                (first && kk == 0) ? 0u : 1u);
+            };
+            bool ok = wait_one(&bars->kv_full, 0) && wait_one(&bars->full[0], 0);
             if (!ok) flag_timeout(p.status, bars);
             ptx::tc_fence_after();
+            if (ok) {
+                issue_sdp(0, 0);
+                issue_sdp(0, 1);
+            }
             for (int i = 0; i < nq && ok; ++i) {
-                const int st = i % kDkvStages;
-                const uint32_t aQ = aRing + (2 * st) * kTile, aDO = aRing + (2 * st + 1) * kTile;
-                ok = wait_one(&bars->full[st], (i / kDkvStages) & 1);
-                if (!ok) {
-                    flag_timeout(p.status, bars);
-                    break;
+                const int st = i % kDkvStages, st2 = (i + 1) % kDkvStages;
+                const bool next = i + 1 < nq;
+                for (int h = 0; h < 2; ++h) {
+                    if (!wait_one(p_ready[h], i & 1)) {
+                        flag_timeout(p.status, bars);
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    issue_pv(st, h, i == 0 && h == 0);
+                    if (h == 1) ptx::mma_commit(&bars->empty[st]);  // Q, dO of tile i are read
+                    if (next) {
+                        if (h == 0) {
+                            if (!wait_one(&bars->full[st2], ((i + 1) / kDkvStages) & 1)) {
+                                flag_timeout(p.status, bars);
+                                ok = false;
+                                break;
+                            }
+                            ptx::tc_fence_after();
+                        }
+                        issue_sdp(st2, h);
+                    }
                 }
-                ptx::tc_fence_after();
-                const uint64_t dQk = kdesc(aQ), dOk = kdesc(aDO), dQm = mndesc(aQ), dOm = mndesc(aDO);
-#pragma unroll
-                for (int k = 0; k < kD / 16; ++k) ptx::mma_ss(tmem + 0, dK + koff(k), dQk + koff(k), idesc_ss, k > 0);
-#pragma unroll
-                for (int k = 0; k < kD / 16; ++k) ptx::mma_ss(tmem + 128, dV + koff(k), dOk + koff(k), idesc_ss, k > 0);
-                ptx::mma_commit(&bars->s_full);
-                if (!wait_one(&bars->p_full, i & 1)) {
-                    flag_timeout(p.status, bars);
-                    ok = false;
-                    break;
-                }
-                ptx::tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < 128 / 16; ++k)
-                    ptx::mma_ts(tmem + 256, tmem + 0 + acol(k), dOm + mnoff(k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-                for (int k = 0; k < 128 / 16; ++k)
-                    ptx::mma_ts(tmem + 384, tmem + 128 + acol(k), dQm + mnoff(k), idesc_ts, (i > 0 || k > 0) ? 1u : 0u);
-                ptx::mma_commit(&bars->empty[st]);
             }
             if (ok) ptx::mma_commit(&bars->fin);
             ptx::mma_commit(&bars->drain);
@@ -291,8 +331,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
         __syncwarp();
     } else {
         // ------------------------------------------------------ compute warps
-        // Column half hs: query columns 64hs .. 64hs+63 of S^T / dP^T, and
-        // feature columns 64hs .. of dV / dK in the epilogue.
+        // Half hs: query rows 64hs .. 64hs+63 of every tile (its own S^T /
+        // dP^T columns 128hs ..), and feature columns 64hs .. of dV / dK in
+        // the epilogue.
         const int hs = warp / 4;
         const int r = (warp % 4) * 32 + lane;  // TMEM lane
         const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
@@ -330,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
                 st_D[64 * hs + r] = nD;
                 if (i + 1 < nq) load_stat(i + 1, nl2, nD);
             }
-            const bool got = ptx::mbar_wait(&bars->s_full, i & 1, p.wait_limit, abort_flag);
+            const bool got = ptx::mbar_wait(hs ? &bars->dp_full : &bars->s_full, i & 1, p.wait_limit, abort_flag);
             if (!half_all(hs, got)) {  // also publishes this half's st_lse / st_D
                 flag_timeout(p.status, bars);
                 ok = false;
@@ -349,18 +390,18 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
                 lo_r = j > tq0 ? (j - tq0) << gshift : 0;
                 hi_r = 128;
             }
+            const uint32_t tH = tmem + lane_off + 128 * hs;  // this half's S^T | dP^T
 #pragma unroll 1
             for (int c = 0; c < 2; ++c) {
-                const int col = 64 * hs + 32 * c;  // first query column of the chunk
                 uint32_t sr[32], dr[32];
-                ptx::tmem_ld32(tmem + lane_off + 0 + col, sr);
-                ptx::tmem_ld32(tmem + lane_off + 128 + col, dr);
+                ptx::tmem_ld32(tH + 32 * c, sr);
+                ptx::tmem_ld32(tH + 64 + 32 * c, dr);
                 ptx::tmem_wait_ld();
                 uint32_t pp[16], dd[16];
 #pragma unroll
                 for (int e2 = 0; e2 < 16; ++e2) {
                     float pv[2], dv[2];
-                    const int r0 = col + 2 * e2;
+                    const int r0 = 64 * hs + 32 * c + 2 * e2;  // query row of the tile
                     const float2 ex = exp2_pair(make_float2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -st_lse[r0]),
                                                             fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -st_lse[r0 + 1])),
                                                 e2);
@@ -375,14 +416,14 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
                     pp[e2] = ptx::pack_bf16x2(pv[0], pv[1]);
                     dd[e2] = ptx::pack_bf16x2(dv[0], dv[1]);
                 }
-                // chunk c's packed columns [64hs + 16c, +16) lie in this
-                // half's columns that this thread has already read
-                ptx::tmem_st16(tmem + lane_off + 0 + 64 * hs + 16 * c, pp);
-                ptx::tmem_st16(tmem + lane_off + 128 + 64 * hs + 16 * c, dd);
+                // chunk c's packed columns [16c, 16c+16) lie in columns
+                // this thread has already read
+                ptx::tmem_st16(tH + 16 * c, pp);
+                ptx::tmem_st16(tH + 64 + 16 * c, dd);
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
-            ptx::mbar_arrive(&bars->p_full);
+            ptx::mbar_arrive(hs ? &bars->p_full2 : &bars->p_full);
         }
         if (ok) {
             const bool got = ptx::mbar_wait(&bars->fin, 0, p.wait_limit, abort_flag);
@@ -503,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
     const int n_dep = (nv * p.Ld + kBK - 1) / kBK;
     const int n_items = n_kv + n_dep;
 
-    if (threadIdx.x == 0) init_bars(bars, kDqStages);
+    if (threadIdx.x == 0) init_bars(bars, kDqStages, kComputeThreads);
     if (warp == 0) {
         ptx::tmem_alloc(&bars->tmem_base, 512);
         ptx::tmem_relinquish();
