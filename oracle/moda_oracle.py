@@ -37,7 +37,7 @@ over layers or a dynamic selection): an optional ``depth_sel`` [B, T, Ld] of
 booleans keeps depth entry i of token t only where depth_sel[b,t,i] is true;
 the other depth logits leave the softmax (as if that slot were absent).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
   * the depth logits take the same ``scale`` as the sequence logits (the §1.2
     formula divides the whole concatenation by sqrt(d));
   * GQA maps query head h to kv-head h // G;
