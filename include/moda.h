@@ -62,7 +62,7 @@ extern "C" {
 typedef enum {
     MODA_OK = 0,
     MODA_ERR_INVALID_VALUE = 1,   /* NULL pointer, non-positive size, Hq % Hkv != 0 */
-    MODA_ERR_UNSUPPORTED = 2,     /* valid shape this build does not implement      */
+    MODA_ERR_UNSUPPORTED = 2,     /* valid shape the library does not implement     */
     MODA_ERR_MISALIGNED = 3,      /* a tensor pointer is not 16-byte aligned         */
     MODA_ERR_WORKSPACE = 4,       /* workspace NULL or smaller than required         */
     MODA_ERR_LAUNCH = 5,          /* the CUDA launch (or tensor-map encode) failed   */
@@ -76,7 +76,7 @@ typedef enum { MODA_BF16 = 0, MODA_F32 = 1 } moda_dtype;
  * tensor-core path when the shape supports it, else SIMT. */
 typedef enum { MODA_IMPL_AUTO = 0, MODA_IMPL_SIMT = 1, MODA_IMPL_TC = 2 } moda_impl;
 
-/* Version of this ABI (MODA_ABI_VERSION of the build). */
+/* Version of this ABI (MODA_ABI_VERSION of the library). */
 int moda_abi_version(void);
 
 /* Human-readable name of a status code. Never NULL; static storage. */
