@@ -6,9 +6,13 @@ attention) on B200.
 
 One step = one MoDA forward over the 64K long-context workload (B=1,
 T=65536, Hq=32, Hkv=4, d=128, Ld=28, bf16, seeded N(0,1) inputs) with inputs
-resident in HBM. N>1 runs N independent replicas (one process per GPU, no
-data-path collective; the barrier and the max-over-ranks timing use NCCL).
-Rank 0 prints one JSON line.
+resident in HBM. With N > 1 GPUs (launched by torchrun, or by this script
+itself when started as ``python bench.py --gpus N``) every rank is one
+process on its own GPU: ``--partition replicas`` (default) runs the whole
+workload on every rank (weak scaling); ``--partition heads`` gives rank r the
+kv-heads [r*Hkv/N, (r+1)*Hkv/N) and their query heads (strong scaling: the
+path needs no exchange across (b, kv-head)). NCCL carries only the barrier
+and the max-over-ranks time. Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -104,10 +108,17 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------- timing
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, cpu_only: bool = False):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if cpu_only:
+        if world > 1:
+            import datetime
+
+            import torch.distributed as dist
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        return world, rank, local
     if world > 1:
         import datetime
 
@@ -160,6 +171,33 @@ def timed(fn, steps, warmup, world, per_launch=True):
     total = t0.elapsed_time(t1) / steps
     launch = statistics.mean(a.elapsed_time(b) for a, b in evs)
     return max_over_ranks(total, world), launch
+
+
+def timed_interleaved(fns, steps_each, warmup, world, block=5):
+    """Interleaved timing of several step functions: rounds of ``block`` calls
+    of each function in turn (A x block, B x block, A x block, ...), so that
+    slow drifts (clocks, power) hit every arm alike. Returns, per function,
+    the max-over-ranks mean ms per call over ``steps_each`` calls."""
+    for fn in fns:
+        for _ in range(warmup):
+            fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    stream = torch.cuda.current_stream()
+    rounds = max(1, (steps_each + block - 1) // block)
+    evs = [[] for _ in fns]
+    for _ in range(rounds):
+        for i, fn in enumerate(fns):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(block):
+                fn()
+            b.record(stream)
+            evs[i].append((a, b))
+    torch.cuda.synchronize()
+    barrier(world)
+    return [max_over_ranks(sum(a.elapsed_time(b) for a, b in e) / (rounds * block), world)
+            for e in evs]
 
 
 # --------------------------------------------------------------- cpu oracle
@@ -274,43 +312,60 @@ def make_step(moda, w, x, mode, kernel, depth_sel=None):
                       impl=kernel)
         moda.moda_bwd(x["q"], x["k"], x["v"], x["kd"], x["vd"], out, lse, x["dout"], w.scale,
                       grads=grads, workspace=ws, impl=kernel)
-    # forward 1; backward: D, depth dq, depth dk/dv (Ld > 0), sequence, 3 conversions
-    return step, 1 + 6 + (1 if w.Ld else 0), out, lse
+    # forward 1; tensor-core backward: D~, dq, dk/dv, depth dk/dv (Ld > 0),
+    # 2 conversions; SIMT backward: D~, dq, dk/dv, depth (Ld > 0)
+    bwd = (3 if kernel == "simt" else 5) + (1 if w.Ld else 0)
+    return step, 1 + bwd, out, lse
 
 
-def measure_secondary(moda, w, world, kernel, steps=5, warmup=3):
-    """Forward TFLOP/s and overhead vs Ld = 0 of another workload; for the
-    forward+backward workload also the backward time and fwd+bwd TFLOP/s."""
+def measure_secondary(moda, w, world, kernel, steps=20, warmup=3):
+    """Forward TFLOP/s and overhead vs Ld = 0 of another workload (the two
+    arms interleaved, ``steps`` calls each); for the forward+backward
+    workload also the backward time and fwd+bwd TFLOP/s."""
     x = {k: v.cuda() for k, v in make_inputs(w, with_dout=w.backward).items()}
     step, _, out, lse = make_step(moda, w, x, "fwd", kernel)
-    ms, _ = timed(step, steps, warmup, world)
     x0 = dict(x, kd=None, vd=None)
     w0 = w.with_(Ld=0)
     step0, _, _, _ = make_step(moda, w0, x0, "fwd", kernel)
-    ms0, _ = timed(step0, steps, warmup, world)
+    ms, ms0 = timed_interleaved([step, step0], steps, warmup, world)
     res = {"config": f"B={w.B} T={w.T} Hq={w.Hq} Hkv={w.Hkv} d={w.d} Ld={w.Ld}",
            "fwd_ms": ms, "fwd_tflops": credited_flops(w) / (ms * 1e-3) / 1e12,
-           "ld0_fwd_ms": ms0, "overhead_vs_ld0": ms / ms0 - 1.0}
+           "ld0_fwd_ms": ms0, "overhead_vs_ld0": ms / ms0 - 1.0,
+           "depth_stream_gbs": depth_stream_gbs(w, ms, ms0),
+           "timing": f"Ld and Ld=0 arms interleaved in blocks of 5, {steps} calls each"}
     # Selected depth: each token keeps a window of its most recent slots
     # (width uniform in [0, Ld]), the same FLOPs are issued (whole tiles).
     sel = pack_depth_sel(make_depth_sel(w, "window")).cuda() if w.Ld else None
     if sel is not None:
         steps_sel, _, _, _ = make_step(moda, w, x, "fwd", kernel, depth_sel=sel)
-        mss, _ = timed(steps_sel, steps, warmup, world)
-        res.update({"sel_window_fwd_ms": mss, "sel_vs_all_slots": mss / ms - 1.0})
+        ms_a, mss = timed_interleaved([step, steps_sel], steps, warmup, world)
+        res.update({"sel_window_fwd_ms": mss, "sel_vs_all_slots": mss / ms_a - 1.0})
     if w.backward:
         stepb, _, _, _ = make_step(moda, w, x, "fwdbwd", kernel)
-        msb, _ = timed(stepb, steps, warmup, world)
-        res.update({"fwd_bwd_ms": msb, "bwd_ms": msb - ms,
-                    "bwd_tflops": 2.5 * credited_flops(w) / ((msb - ms) * 1e-3) / 1e12,
+        ms_f, msb = timed_interleaved([step, stepb], steps, warmup, world)
+        res.update({"fwd_bwd_ms": msb, "bwd_ms": msb - ms_f,
+                    "bwd_tflops": 2.5 * credited_flops(w) / ((msb - ms_f) * 1e-3) / 1e12,
                     "fwd_bwd_tflops": 3.5 * credited_flops(w) / (msb * 1e-3) / 1e12})
         if sel is not None:
             stepbs, _, _, _ = make_step(moda, w, x, "fwdbwd", kernel, depth_sel=sel)
-            msbs, _ = timed(stepbs, steps, warmup, world)
-            res.update({"sel_window_fwd_bwd_ms": msbs, "sel_fwd_bwd_vs_all_slots": msbs / msb - 1.0})
+            msb2, msbs = timed_interleaved([stepb, stepbs], steps, warmup, world)
+            res.update({"sel_window_fwd_bwd_ms": msbs, "sel_fwd_bwd_vs_all_slots": msbs / msb2 - 1.0})
     del x
     torch.cuda.empty_cache()
     return res
+
+
+def depth_stream_bytes(w) -> int:
+    """Algorithmic bytes of the depth stream: kd and vd read once."""
+    return 2 * w.B * w.T * w.Ld * w.Hkv * w.d * (2 if w.dtype == "bf16" else 4)
+
+
+def depth_stream_gbs(w, ms, ms0):
+    """Depth-stream bandwidth as the time the depth keys add: bytes(kd + vd)
+    / (t(Ld) - t(Ld=0)); None when the difference is not positive (the depth
+    work hidden within run-to-run noise)."""
+    dt = (ms - ms0) * 1e-3
+    return depth_stream_bytes(w) / dt / 1e9 if dt > 0 else None
 
 
 def code_hash(path: str) -> str:
@@ -337,6 +392,70 @@ def traffic_for(kernel_src: str):
     return t.get("dram_bytes_per_launch")
 
 
+def relaunch_under_torchrun(argv, n_gpus: int) -> int:
+    """``python bench.py --gpus N`` outside torchrun: start N ranks (one
+    process per GPU) under torch.distributed.run on this node and return its
+    exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n_gpus}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + list(argv)
+    return subprocess.call(cmd)
+
+
+def shard_heads(w, x, rank: int, world: int):
+    """Rank ``rank``'s share under head partitioning: kv-heads
+    [rank*Hkv/world, (rank+1)*Hkv/world) and their G query heads each, as
+    contiguous tensors (what a head-parallel layer holds). No exchange is
+    needed: each GQA group's output depends only on its own q, k, v, kd, vd."""
+    if w.Hkv % world:
+        raise SystemExit(f"--partition heads needs the world size ({world}) to divide Hkv={w.Hkv}")
+    hk = w.Hkv // world
+    g0, g1 = rank * hk, (rank + 1) * hk
+    q0, q1 = g0 * w.G, g1 * w.G
+    xs = {"q": x["q"][:, :, q0:q1], "k": x["k"][:, :, g0:g1], "v": x["v"][:, :, g0:g1],
+          "kd": x["kd"][:, :, :, g0:g1], "vd": x["vd"][:, :, :, g0:g1]}
+    if "dout" in x:
+        xs["dout"] = x["dout"][:, :, q0:q1]
+    return w.with_(name=f"{w.name}-heads{g0}-{g1}", Hq=q1 - q0, Hkv=hk), \
+        {k: v.contiguous() for k, v in xs.items()}
+
+
+def dry_run(args, w) -> int:
+    """``--dry-run``: the rank plumbing without a GPU. Ranks join over gloo,
+    each takes its partition of the workload (shapes only, nothing timed),
+    the shares are gathered and rank 0 prints one JSON line with the plan."""
+    import torch.distributed as dist
+    world, rank, _ = dist_setup(args.gpus, cpu_only=True)
+    if args.partition == "heads" and world > 1:
+        if w.Hkv % world:
+            raise SystemExit(f"--partition heads needs the world size ({world}) to divide Hkv={w.Hkv}")
+        hk = w.Hkv // world
+        share = {"rank": rank, "kv_heads": [rank * hk, (rank + 1) * hk],
+                 "q_heads": [rank * hk * w.G, (rank + 1) * hk * w.G],
+                 "flops": credited_flops(w.with_(Hq=hk * w.G, Hkv=hk))}
+    else:
+        share = {"rank": rank, "kv_heads": [0, w.Hkv], "q_heads": [0, w.Hq],
+                 "flops": credited_flops(w)}
+    shares = [None] * world
+    if world > 1:
+        dist.all_gather_object(shares, share)
+        barrier(world)
+    else:
+        shares = [share]
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "n_gpus": world, "partition": args.partition,
+                          "workload": w.name, "job_flops": sum(x["flops"] for x in shares),
+                          "full_flops": credited_flops(w),
+                          "scaling": "weak" if args.partition == "replicas" else "strong",
+                          "shares": shares}), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -345,29 +464,44 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="t64k", choices=sorted(WORKLOADS))
     ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--partition", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: every rank runs the whole workload (replicas, weak scaling) "
+                         "or its share of the kv-heads (heads, strong scaling)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--no-extra", action="store_true", help="skip the Ld=0 and e2e runs")
+    ap.add_argument("--extra-steps", type=int, default=20,
+                    help="calls per arm of the interleaved overhead / pack / secondary timings")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the Ld=0, pack, e2e and secondary-workload runs")
     ap.add_argument("--mode", default="fwd", choices=["fwd", "fwdbwd"],
                     help="step = forward, or forward + backward (credited 3.5x the forward FLOPs)")
     ap.add_argument("--shape", default=None,
                     help="B,T,Hq,Hkv,d,Ld override of the workload (profiling runs)")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="no GPU: start the ranks (gloo), print the partition plan, time nothing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ and args.impl == "ours":
+        return relaunch_under_torchrun(sys.argv[1:], args.gpus)
     w = WORKLOADS[args.workload]
     if args.shape:
         B, T, Hq, Hkv, d, Ld = (int(v) for v in args.shape.split(","))
         w = w.with_(name=f"{w.name}-shape", B=B, T=T, Hq=Hq, Hkv=Hkv, d=d, Ld=Ld)
     if args.impl == "reference":
         return reference_arm(args, w)
+    if args.dry_run:
+        return dry_run(args, w)
 
     import depth_kv_attention_b200 as moda
 
     world, rank, local = dist_setup(args.gpus)
     peaks, peaks_kind = load_peaks()
+    w_full = w
     x_host = make_inputs(w, with_dout=args.mode == "fwdbwd")
+    if args.partition == "heads" and world > 1:
+        w, x_host = shard_heads(w, x_host, rank, world)
     x = {k: v.cuda() for k, v in x_host.items()}
     step, launches_per_step, out, lse = make_step(moda, w, x, args.mode, args.kernel)
 
@@ -379,52 +513,89 @@ def main():
     clocks.start()
     ms, launch_ms = timed(step, args.steps, args.warmup, world)
     clk = clocks.stop()
-    flops = credited_flops(w) * (3.5 if args.mode == "fwdbwd" else 1.0)
-    value = flops * world / (ms * 1e-3) / 1e12
-
+    mult = 3.5 if args.mode == "fwdbwd" else 1.0
+    flops_rank = credited_flops(w) * mult
+    # whole-job work: every replica's, or the one workload split over ranks
+    flops_job = credited_flops(w_full) * mult * (world if args.partition == "replicas" else 1)
+    value = flops_job / (ms * 1e-3) / 1e12
     extra = {}
     if not args.no_extra and args.mode == "fwd" and not args.shape:
-        # the same library's own causal attention with Ld = 0
+        # the same library's own causal attention with Ld = 0, interleaved
+        # with the Ld forward; the difference gives the depth stream's rate
         out0 = torch.empty_like(out)
+        lse0 = torch.empty_like(lse)
 
         def step0():
-            moda.moda_fwd(x["q"], x["k"], x["v"], None, None, w.scale, out=out0, lse=lse,
+            moda.moda_fwd(x["q"], x["k"], x["v"], None, None, w.scale, out=out0, lse=lse0,
                           impl=args.kernel)
-        ms0, _ = timed(step0, args.steps, args.warmup, world)
+        ms_a, ms0 = timed_interleaved([step, step0], args.extra_steps, args.warmup, world)
         extra["ld0_ms_per_step"] = ms0
-        extra["overhead_vs_ld0"] = ms / ms0 - 1.0
-        del out0
+        extra["overhead_vs_ld0"] = ms_a / ms0 - 1.0
+        extra["overhead_timing"] = (f"Ld={w.Ld} and Ld=0 forwards interleaved in blocks of 5, "
+                                    f"{args.extra_steps} calls each ({ms_a:.3f} vs {ms0:.3f} ms)")
+        extra["depth_stream_gbs"] = depth_stream_gbs(w, ms_a, ms0)
+        extra["depth_stream_bytes"] = depth_stream_bytes(w)
+        del out0, lse0
+        # the optional repack: moda_pack_depth + moda_fwd_packed against the
+        # forward on the native depth layout
+        packed = moda.moda_pack_depth(x["kd"], x["vd"])
+        outp = torch.empty_like(out)
+
+        def step_pack():
+            moda.moda_pack_depth(x["kd"], x["vd"], packed=packed)
+
+        def step_fwd_packed():
+            moda.moda_fwd_packed(x["q"], x["k"], x["v"], packed, w.Ld, w.scale, out=outp, lse=lse)
+
+        def step_pack_fwd():
+            step_pack()
+            step_fwd_packed()
+        ms_n, ms_p, ms_fp, ms_pf = timed_interleaved([step, step_pack, step_fwd_packed, step_pack_fwd],
+                                                     args.extra_steps, args.warmup, world)
+        extra["pack_depth"] = {
+            "t_fwd_native_ms": ms_n, "t_pack_ms": ms_p, "t_fwd_packed_ms": ms_fp,
+            "t_pack_plus_fwd_packed_ms": ms_pf, "pack_vs_native": ms_pf / ms_n - 1.0,
+            "pack_gbs": 2 * depth_stream_bytes(w) / (ms_p * 1e-3) / 1e9,
+            "timing": f"four arms interleaved in blocks of 5, {args.extra_steps} calls each"}
+        del packed, outp
+        torch.cuda.empty_cache()
 
     e2e = None
     if not args.no_extra and args.mode == "fwd":
         pinned = {k: v.pin_memory() for k, v in x_host.items()}
         out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-        bufs = dict(x, out=out, lse=lse)
+        staging = torch.empty(moda.moda_fwd_host_staging_bytes(w.B, w.T, w.Hq, w.Hkv, w.d, w.Ld,
+                                                                x_host["q"].dtype),
+                              dtype=torch.uint8, device="cuda")
 
         def step_e2e():
             moda.moda_fwd_from_host(pinned["q"], pinned["k"], pinned["v"], pinned["kd"], pinned["vd"],
-                                    w.scale, out_host=out_h, lse_host=lse_h, dev_bufs=bufs,
-                                    impl=args.kernel)
+                                    w.scale, out_host=out_h, lse_host=lse_h, staging=staging)
         ms_e2e, _ = timed(step_e2e, args.e2e_steps, 3, world)
         h2d = sum(v.numel() * v.element_size() for v in pinned.values())
         d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
-        e2e = {"value": flops * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+        e2e = {"value": flops_job / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+               "api": "moda_fwd_host (C ABI): pinned host inputs -> device staging -> forward -> "
+                      "out, lse to pinned host, then a stream synchronize"}
+        del staging
+        torch.cuda.empty_cache()
 
     kernel_src = os.path.join(ROOT, "depth_kv_attention_b200", "csrc",
                               "moda_simt.cu" if args.kernel == "simt" else "moda_fwd_sm100.cu")
     peak = peaks["bf16_tflops"]
-    achieved = flops / (launch_ms * 1e-3) / 1e12
+    achieved = flops_rank / (launch_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic_for(kernel_src),
                 "peak_kind": f"{peaks_kind} bf16 burst (cuBLAS 8192^3)",
                 "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                 "frac_of_nominal_2250": achieved / 2250.0}
 
-    if not args.no_extra and not args.shape:
-        extra["other_workloads"] = {name: measure_secondary(moda, WORKLOADS[name], world, args.kernel)
-                                    for name in ("t4k", "t16k_b2", "g32_fwdbwd") if name != w.name}
+    if not args.no_extra and not args.shape and args.partition == "replicas":
+        extra["other_workloads"] = {
+            name: measure_secondary(moda, WORKLOADS[name], world, args.kernel, steps=args.extra_steps)
+            for name in ("t4k", "t16k_b2", "g32_fwdbwd") if name != w.name}
 
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0 and args.mode == "fwd":
@@ -434,12 +605,17 @@ def main():
                          f"of the same workload, {secs:.1f} s, credited FLOPs 4*d*(t+1+Ld) per row"}
 
     if rank == 0:
+        cfg = workload_config(w_full)
+        cfg["parallelism"] = (f"replicas x{world}" if args.partition == "replicas"
+                              else f"kv-head shards x{world}")
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": workload_config(w),
-            "pct_of_bf16_peak": 100.0 * value / world / peak,
+            "higher_is_better": True,
+            "scaling": "weak" if args.partition == "replicas" else "strong",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": cfg,
+            "pct_of_bf16_peak": 100.0 * achieved / peak,
             "clocks": clk, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
             "roofline": roofline, "cpu_baseline": cpu, "kernel_family": args.kernel,
             "mode": args.mode,

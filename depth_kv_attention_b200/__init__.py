@@ -22,6 +22,7 @@ __all__ = [
     "moda_fwd", "moda_fwd_sel", "moda_bwd", "moda_bwd_sel", "moda_bwd_workspace_bytes", "moda_bwd_noalloc", "moda_pack_depth",
     "moda_pack_depth_bytes", "moda_fwd_packed", "moda_depth_write", "moda_device_status",
     "moda_debug_set_wait_limit", "moda_debug_exp2_poly", "moda_fwd_from_host",
+    "moda_fwd_host_staging_bytes",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoda.so")
@@ -62,6 +63,8 @@ _c_dev_status = _sig("moda_device_status", _i, [_vp])
 _c_wait_limit = _sig("moda_debug_set_wait_limit", _i, [ctypes.c_uint32])
 _c_exp2_poly = _sig("moda_debug_exp2_poly", _i, [_vp, _vp, _i, _vp])
 _c_bwd_noalloc = _sig("moda_bwd_noalloc", _i, [_vp] * 8 + _DIMS + [_i, _f] + [_vp] * 5 + [_vp])
+_c_host_bytes = _sig("moda_fwd_host_staging_bytes", _sz, _DIMS + [_i])
+_c_fwd_host = _sig("moda_fwd_host", _i, [_vp] * 5 + _DIMS + [_i, _f, _vp, _vp, _vp, _sz, _vp])
 
 
 class ModaError(RuntimeError):
@@ -313,32 +316,41 @@ def moda_debug_exp2_poly(x, y=None, stream=None):
     return y
 
 
+def moda_fwd_host_staging_bytes(B, T, Hq, Hkv, d, Ld, dtype) -> int:
+    return _c_host_bytes(B, T, Hq, Hkv, d, Ld, _DTYPE[dtype])
+
+
 def moda_fwd_from_host(q, k, v, kd=None, vd=None, scale: float | None = None, device="cuda",
-                       out_host=None, lse_host=None, dev_bufs=None, impl: str = "auto"):
-    """End-to-end forward from HOST tensors: copy inputs host->device on the
-    current stream, run ``moda_fwd``, copy out and lse back to host buffers.
+                       out_host=None, lse_host=None, staging=None, stream=None):
+    """End-to-end forward from HOST tensors through ``moda_fwd_host``: the C
+    call enqueues the host->device copies of the inputs into the device
+    ``staging`` buffer, the forward and the device->host copies of out and
+    lse; this function then waits for the stream.
 
     ``out_host`` / ``lse_host`` (pinned CPU tensors) are filled in place when
-    given. ``dev_bufs`` may hold pre-allocated device buffers
-    (q,k,v,kd,vd,out,lse) to keep allocation out of a timed loop.
-    Returns (out_host, lse_host) after the stream has finished.
-    """
-    B, T, Hq, d = q.shape
-    if dev_bufs is None:
-        dev_bufs = {n: (None if t is None else torch.empty(t.shape, dtype=t.dtype, device=device))
-                    for n, t in dict(q=q, k=k, v=v, kd=kd, vd=vd).items()}
-        dev_bufs["out"] = torch.empty(q.shape, dtype=q.dtype, device=device)
-        dev_bufs["lse"] = torch.empty((B, Hq, T), dtype=torch.float32, device=device)
-    for n, t in dict(q=q, k=k, v=v, kd=kd, vd=vd).items():
-        if t is not None:
-            dev_bufs[n].copy_(t, non_blocking=True)
-    moda_fwd(dev_bufs["q"], dev_bufs["k"], dev_bufs["v"], dev_bufs["kd"], dev_bufs["vd"], scale,
-             out=dev_bufs["out"], lse=dev_bufs["lse"], impl=impl)
+    given, else created (pinned). ``staging`` (a CUDA uint8 tensor of at
+    least ``moda_fwd_host_staging_bytes`` bytes) is created when not given.
+    Returns (out_host, lse_host)."""
+    if kd is not None and kd.shape[2] == 0:
+        kd = vd = None
+    for t in (q, k, v, kd, vd, out_host, lse_host):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError("moda_fwd_from_host takes contiguous host tensors")
+    B, T, Hq, Hkv, d, Ld = _dims(q, k, kd)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dev = torch.device(device)
+    need = moda_fwd_host_staging_bytes(B, T, Hq, Hkv, d, Ld, q.dtype)
+    if staging is None:
+        staging = torch.empty(need, dtype=torch.uint8, device=dev)
     if out_host is None:
         out_host = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
     if lse_host is None:
         lse_host = torch.empty((B, Hq, T), dtype=torch.float32, pin_memory=True)
-    out_host.copy_(dev_bufs["out"], non_blocking=True)
-    lse_host.copy_(dev_bufs["lse"], non_blocking=True)
-    torch.cuda.current_stream().synchronize()
+    with torch.cuda.device(staging.device):
+        st = _stream(stream)
+        _check(_c_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(kd), _ptr(vd), B, T, Hq, Hkv, d, Ld,
+                           _DTYPE[q.dtype], scale, _ptr(out_host), _ptr(lse_host), _ptr(staging),
+                           staging.numel(), st), "moda_fwd_host")
+        _check(_c_dev_status(st), "moda_fwd_host (stream)")
     return out_host, lse_host

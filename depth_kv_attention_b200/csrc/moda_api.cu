@@ -1,10 +1,13 @@
 // Host side of the C ABI declared in include/moda.h: argument validation,
 // kernel-family selection and launch. No allocation, no synchronisation
-// (except moda_device_status), no state beyond the device status word.
+// (except moda_device_status), no state beyond the device status word and
+// the test hook's wait limit.
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
 #include "moda_internal.h"
+#include "symbol_addr.h"
 
 namespace moda {
 
@@ -15,24 +18,21 @@ __device__ unsigned int g_status_word;
 namespace {
 
 constexpr int kMaxDevices = 64;
-unsigned int* g_status_ptr[kMaxDevices];
-unsigned int g_wait_limit[kMaxDevices];
+SymbolAddr g_status_addr(&g_status_word);
+std::atomic<unsigned int> g_wait_limit[kMaxDevices];
 
-// Device address of the status word on the current device (resolved once per
-// device; cudaGetSymbolAddress needs the device current).
+// Device address of the status word in the current context (resolved per
+// context, see symbol_addr.h) and the wait limit set for this device.
 cudaError_t status_ptr(unsigned int** p, unsigned int* wait_limit) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    if (!g_status_ptr[dev]) {
-        void* a = nullptr;
-        e = cudaGetSymbolAddress(&a, g_status_word);
-        if (e != cudaSuccess) return e;
-        g_status_ptr[dev] = static_cast<unsigned int*>(a);
-    }
-    *p = g_status_ptr[dev];
-    if (wait_limit) *wait_limit = g_wait_limit[dev];
+    void* a = nullptr;
+    e = g_status_addr.get(&a);
+    if (e != cudaSuccess) return e;
+    *p = static_cast<unsigned int*>(a);
+    if (wait_limit) *wait_limit = g_wait_limit[dev].load(std::memory_order_relaxed);
     return cudaSuccess;
 }
 
@@ -99,6 +99,22 @@ size_t bwd_ws_rowD_bytes(int B, int T, int Hq) {
 size_t bwd_ws_bytes(int B, int T, int Hq, int Hkv, int d, bool with_acc) {
     size_t acc = with_acc ? (size_t)B * T * 2 * Hkv * d * sizeof(float) : 0;
     return bwd_ws_rowD_bytes(B, T, Hq) + acc;
+}
+
+// Staging layout of moda_fwd_host: q, k, v, kd, vd, out, lse, each at a
+// 256-byte-aligned offset. Returns the total size; offs[] receives offsets.
+size_t host_staging_layout(int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dt, size_t offs[7]) {
+    const size_t esz = dt == MODA_F32 ? 4 : 2;
+    const size_t n[7] = {(size_t)B * T * Hq * d * esz, (size_t)B * T * Hkv * d * esz,
+                         (size_t)B * T * Hkv * d * esz, (size_t)B * T * Ld * Hkv * d * esz,
+                         (size_t)B * T * Ld * Hkv * d * esz, (size_t)B * T * Hq * d * esz,
+                         (size_t)B * Hq * T * sizeof(float)};
+    size_t o = 0;
+    for (int i = 0; i < 7; ++i) {
+        offs[i] = o;
+        o += (n[i] + 255) & ~size_t(255);
+    }
+    return o;
 }
 
 }  // namespace
@@ -267,6 +283,54 @@ moda_status moda_fwd_packed(const void* q, const void* k, const void* v, const v
     return run_fwd(a, stream, MODA_IMPL_AUTO);
 }
 
+size_t moda_fwd_host_staging_bytes(int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dtype) {
+    if (check_dims(B, T, Hq, Hkv, d, Ld) != MODA_OK) return 0;
+    if (dtype != MODA_BF16 && dtype != MODA_F32) return 0;
+    size_t offs[7];
+    return host_staging_layout(B, T, Hq, Hkv, d, Ld, dtype, offs);
+}
+
+moda_status moda_fwd_host(const void* q, const void* k, const void* v, const void* kd, const void* vd,
+                          int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dtype, float scale,
+                          void* out, float* lse, void* staging, size_t staging_bytes, void* stream) {
+    moda_status st = check_dims(B, T, Hq, Hkv, d, Ld);
+    if (st != MODA_OK) return st;
+    if (dtype != MODA_BF16 && dtype != MODA_F32) return MODA_ERR_INVALID_VALUE;
+    if (!q || !k || !v || !out) return MODA_ERR_INVALID_VALUE;
+    if (Ld > 0 && (!kd || !vd)) return MODA_ERR_INVALID_VALUE;
+    size_t offs[7];
+    const size_t need = host_staging_layout(B, T, Hq, Hkv, d, Ld, dtype, offs);
+    if (!staging || staging_bytes < need) return MODA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(staging) & 255u) != 0) return MODA_ERR_MISALIGNED;
+    char* base = static_cast<char*>(staging);
+    void* dq = base + offs[0];
+    void* dk = base + offs[1];
+    void* dv = base + offs[2];
+    void* dkd = Ld > 0 ? base + offs[3] : nullptr;
+    void* dvd = Ld > 0 ? base + offs[4] : nullptr;
+    void* dout = base + offs[5];
+    float* dlse = lse ? reinterpret_cast<float*>(base + offs[6]) : nullptr;
+    const size_t esz = dtype == MODA_F32 ? 4 : 2;
+    const size_t nq = (size_t)B * T * Hq * d * esz, nkv = (size_t)B * T * Hkv * d * esz;
+    const size_t ndep = (size_t)B * T * Ld * Hkv * d * esz;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // inputs to the device (one cudaMemcpyAsync per tensor)
+    const void* src[5] = {q, k, v, kd, vd};
+    void* dst[5] = {dq, dk, dv, dkd, dvd};
+    const size_t nb[5] = {nq, nkv, nkv, ndep, ndep};
+    for (int i = 0; i < 5; ++i)
+        if (nb[i] && cudaMemcpyAsync(dst[i], src[i], nb[i], cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return MODA_ERR_CUDA;
+    st = moda_fwd_ex(dq, dk, dv, dkd, dvd, B, T, Hq, Hkv, d, Ld, dtype, scale, dout, dlse, stream,
+                     MODA_IMPL_AUTO);
+    if (st != MODA_OK) return st;
+    if (cudaMemcpyAsync(out, dout, nq, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MODA_ERR_CUDA;
+    if (lse && cudaMemcpyAsync(lse, dlse, (size_t)B * Hq * T * sizeof(float), cudaMemcpyDeviceToHost, s) !=
+                   cudaSuccess)
+        return MODA_ERR_CUDA;
+    return MODA_OK;
+}
+
 moda_status moda_device_status(void* stream) {
     unsigned int* p = nullptr;
     if (status_ptr(&p, nullptr) != cudaSuccess) return MODA_ERR_CUDA;
@@ -293,7 +357,7 @@ moda_status moda_debug_set_wait_limit(uint32_t spins) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MODA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return MODA_ERR_CUDA;
-    g_wait_limit[dev] = spins;
+    g_wait_limit[dev].store(spins, std::memory_order_relaxed);
     return MODA_OK;
 }
 

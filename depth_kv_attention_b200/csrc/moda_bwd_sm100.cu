@@ -3,29 +3,33 @@
 // The pages give no backward pass; this computes the derivative of the MoDA
 // forward ("动态混合深度注意力机制MoDA技术解析" (mhpn.cn) §1.2 formula, §2.2 dual
 // mask) with the usual softmax-Jacobian identities:
-//   P = exp(s - lse),  D = <dout, out>,  dS = P * (dP - D),  dP = dout . v
+//   P = exp(s - lse),  dP = dout . v,  D = sum_j P_j dP_j,  dS = P * (dP - D)
 //   dq = scale (sum_j dS_j k_j + sum_i dS'_i kd_i)
 //   dk_j = scale sum dS_j q,  dv_j = sum P_j dout   (rows t >= j, G heads)
 //   dkd_i = scale sum_h dS'_i q,  dvd_i = sum_h P'_i dout   (same token)
 //
 // Launch sequence (one stream):
-//   1. D = rowsum(dout * out)                      (SIMT, shared with the SIMT path)
-//   2. dk, dv: KV-major tensor-core kernel; partial sums of a key tile over a
-//      chunk of query tiles go to fp32 accumulators with vector reductions
-//   3. dkd, dvd: the same kernel with 128-row depth chunks as the key tiles
+//   1. D~ = rowsum(dout * out), an estimate of D from the stored output (SIMT)
+//   2. dq: query-major tensor-core kernel over the causal key tiles and the
+//      query tile's own depth chunks. It sees all keys of its rows, so it
+//      also forms the exact D = D~ + sum_j P_j (dP_j - D~) and corrects dq
+//      for D - D~; dq accumulates in TMEM and is written once, in bf16
+//   3. dk, dv: KV-major tensor-core kernel (reads the exact D); partial sums
+//      of a key tile over a chunk of query tiles go to fp32 accumulators
+//      with vector reductions
+//   4. dkd, dvd: the same kernel with 128-row depth chunks as the key tiles
 //      and a same-token mask (each depth row owned by one CTA, bf16 stores)
-//   4. dq: query-major tensor-core kernel over the causal key tiles and the
-//      query tile's own depth chunks; dq accumulates in TMEM and is written
-//      once, in bf16 (no dq reductions between CTAs)
 //   5. dk, dv = bf16(accumulators)
-// Splitting dq from dk/dv recomputes S and dP once more (7 instead of 5
-// GEMMs per tile pair) but removes the per-pair fp32 dq reductions, which for
-// wide GQA (G = 32, 4 tokens per 128-row tile) would move gigabytes through L2.
+// Splitting dq from dk/dv recomputes S and dP once more but removes the
+// per-pair fp32 dq reductions, which for wide GQA (G = 32, 4 tokens per
+// 128-row tile) would move gigabytes through L2.
 //
 // Both kernels put query rows in the forward's token-major GQA order (a
-// 128-row tile = n = 128/G tokens x G heads), one warp issues the TMA loads
-// and one the MMAs (whole-warp control, one lane issues), four warps do the
-// elementwise work with one thread per TMEM lane.
+// 128-row tile = n = 128/G tokens x G heads). Warp 8 issues the TMA loads
+// (the whole warp runs the schedule, lane 0 issues), lane 0 of warp 9 issues
+// every tcgen05.mma and commit, and warps 0-7 (two warpgroups, one per
+// 64-column half of every TMEM tile) do the elementwise work, one thread per
+// TMEM lane.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -501,8 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
 struct DqParams {
     CUtensorMap tm_q, tm_do, tm_k, tm_v, tm_kd, tm_vd;
     const float* lse;
-    const float* rowD;
-    void* dq;  // [B,T,Hq,d] bf16
+    float* rowD;  // in: D~ = <dout, out> per row; out: D = sum_j P_j dP_j
+    void* dq;     // [B,T,Hq,d] bf16
     const unsigned long long* depth_sel;  // [B,T] slot masks or null
     int B, T, Hq, Hkv, G, n, Ld, nqt;
     float sl2, scale;
@@ -510,20 +514,45 @@ struct DqParams {
     unsigned int wait_limit;
 };
 constexpr int kDqStages = 4;  // ring of K / V tiles, one per slot
-constexpr int kDqSmem = 2 * kTile + kDqStages * kTile + 256 + 1024;
+constexpr int kDqSmem = 2 * kTile + kDqStages * kTile + 256 + 2 * 128 * 4 + 1024;
 static_assert(kDqSmem <= 232448, "shared memory per CTA");
 
 // One CTA per query tile (n tokens x G heads of one kv group), latest tokens
 // first. Items: the causal key tiles, then the tile's own depth chunks (rows
 // t0*Ld + 128*d .. of the [B, T*Ld, Hkv, d] view, same-token mask).
-// TMEM: R0 | R1 (S and dP alternate between them) | dQ. S(x) sits in
-// R[x % 2] and dP(x) in R[(x + 1) % 2]. Once the compute warps publish
-// dS(x) (written over S(x)), the MMA warp issues, in this order:
+//
+// Row statistic D. The softmax Jacobian needs D_t = sum_j P_tj dP_tj over
+// all keys of row t, which equals <dout, out> only for the exact output: the
+// output the forward stored is rounded to bf16 (and was formed from bf16 P),
+// and wide depth keys amplify that rounding through dq = scale sum dS k by
+// |kd|. This kernel sees every key of its rows, so it computes D itself:
+// with the estimate D~ = <dout, out> (the first kernel of the backward) it
+// forms dS~ = P (dP - D~) in fp32 and accumulates, per row,
+//   delta = sum_j dS~_j   (= D - D~, since sum_j P_j = 1),
+//   dQ~  += dS~ K          (bf16 dS~: the near-cancellation dP - D~ is fp32)
+//   Bq   += P K            (the attention-weighted mean key)
+// and writes dq = scale (dQ~ - delta Bq), i.e. scale sum_j P_j (dP_j - D) k_j,
+// and D = D~ + delta for the dK/dV kernels, which run after this one.
+//
+// Depth items carry dS~ as two bf16 terms, hi = bf16(dS~) and lo =
+// bf16(dS~ - hi) (16 significant bits): depth keys are where MoDA's wide
+// logits live (a token's earlier layers), and there a few large dS~ times
+// large |kd| would otherwise put the bf16 rounding of dS~ (2^-9 relative)
+// straight into dq. It costs 8 MMAs per depth item (one or two per tile).
+//
+// TMEM: R0 | R1 (S and dP alternate between them) | dQ~ | Bq. S(x) sits in
+// R[x % 2] and dP(x) in R[(x + 1) % 2]. The compute warps write P(x) and
+// dS~(x) in bf16 over S(x) (each column half: dS~ at its columns 0-31, P at
+// 32-63; for a depth item the lo term of dS~ over the half's dP columns
+// 0-31, already read); once they publish them the MMA warp issues, in this
+// order (tcgen05.mma operations of one CTA execute in issue order):
 //   S(x+1) = Q K(x+1)^T   into R[(x+1) % 2] (dP(x) there has been read)
-//   dQ    += dS(x) K(x)   A = dS(x) from R[x % 2]
-//   dP(x+1) = dO V(x+1)^T into R[x % 2], after dQ has read dS(x) there
-// so the compute warps exponentiate S(x+1) while dQ and dP(x+1) run, then
-// form dS(x+1) = P (dP - D).
+//   dQ~   += dS~(x) K(x)  A = dS~(x) from R[x % 2]
+//   Bq    += P(x) K(x)    A = P(x) from R[x % 2]
+//   dP(x+1) = dO V(x+1)^T into R[x % 2], after both have read it
+// so the compute warps exponentiate S(x+1) while these run, then form
+// dS~(x+1). A depth item issues dQ~ += lo(x) K(x) (A from R[(x+1) % 2]) after
+// dQ~ and Bq, and S(x+1) only after that.
 __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_constant__ DqParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -531,6 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
     uint8_t* sDO = smem + kTile;
     uint8_t* sRing = smem + 2 * kTile;
     Bars* bars = reinterpret_cast<Bars*>(sRing + kDqStages * kTile);
+    float* sDelta = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // [2 halves][128 rows]
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     volatile int* abort_flag = &bars->abort_flag;
@@ -647,7 +677,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
                     break;
                 }
                 ptx::tc_fence_after();
-                if (x + 1 < n_items && !issue_s(x + 1)) {
+                const bool depth_item = x >= n_kv;
+                if (!depth_item && x + 1 < n_items && !issue_s(x + 1)) {
                     ok = false;
                     break;
                 }
@@ -657,10 +688,24 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
                 for (int k = 0; k < kBK / 16; ++k)
                     ptx::mma_ts(tmem + 256, tmem + (x & 1) * 128 + acol(k), km + mnoff(k), idesc_ts,
                                      (x > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                for (int k = 0; k < kBK / 16; ++k)
+                    ptx::mma_ts(tmem + 384, tmem + (x & 1) * 128 + 32 + acol(k), km + mnoff(k), idesc_ts,
+                                     (x > 0 || k > 0) ? 1u : 0u);
+                if (depth_item) {
+                    // the lo term of dS~(x), then S(x + 1) over it
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        ptx::mma_ts(tmem + 256, tmem + ((x + 1) & 1) * 128 + acol(k), km + mnoff(k), idesc_ts, 1u);
+                    if (x + 1 < n_items && !issue_s(x + 1)) {
+                        ok = false;
+                        break;
+                    }
+                }
                 // K(x), V(x) are no longer needed
                 ptx::mma_commit(&bars->empty[sk % kDqStages]);
                 ptx::mma_commit(&bars->empty[(sk + 1) % kDqStages]);
-                // dP(x + 1) into R[x % 2], after dQ has read dS(x) there
+                // dP(x + 1) into R[x % 2], after dQ~ and Bq have read it
                 if (x + 1 < n_items && !issue_dp(x + 1)) {
                     ok = false;
                     break;
@@ -692,6 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
         const bool has_sel = p.depth_sel != nullptr;
         const unsigned long long sel =
             has_sel && row_ok ? p.depth_sel[(long long)b * p.T + t] & depth_slot_bits(p.Ld) : 0ull;
+        float delta = 0.f;  // sum of this half's dS~ over every item (fp32)
         bool ok = true;
         for (int x = 0; x < n_items; ++x) {
             const uint32_t rS = tmem + lane_off + (x & 1) * 128;        // S(x), then dS(x)
@@ -723,6 +769,14 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
                     pr[c] = ((vw[c >> 5] >> (c & 31)) & 1u) ? e.x : 0.f;
                     pr[c + 1] = ((vw[c >> 5] >> ((c + 1) & 31)) & 1u) ? e.y : 0.f;
                 }
+                // P in bf16 over this half's S columns 32-63 (already read)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t pp[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pp[e] = ptx::pack_bf16x2(pr[32 * c + 2 * e], pr[32 * c + 2 * e + 1]);
+                    ptx::tmem_st16(rS + 64 * hs + 32 + 16 * c, pp);
+                }
             }
             if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->dp_full, x & 1, p.wait_limit, abort_flag))) {
                 flag_timeout(p.status, bars);
@@ -730,19 +784,26 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
                 break;
             }
             ptx::tc_fence_after();
+            const bool depth_item = x >= n_kv;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t dr[32];
                 ptx::tmem_ld32(rP + 64 * hs + 32 * c, dr);
                 ptx::tmem_wait_ld();
-                uint32_t dd[16];
+                uint32_t dd[16], dl[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const float d0 = pr[32 * c + 2 * e] * (__uint_as_float(dr[2 * e]) - Drow);
                     const float d1 = pr[32 * c + 2 * e + 1] * (__uint_as_float(dr[2 * e + 1]) - Drow);
+                    delta += d0 + d1;
                     dd[e] = ptx::pack_bf16x2(d0, d1);
+                    // lo term: the part of dS~ the bf16 hi term drops
+                    dl[e] = ptx::pack_bf16x2(d0 - __uint_as_float(dd[e] << 16),
+                                             d1 - __uint_as_float(dd[e] & 0xffff0000u));
                 }
                 ptx::tmem_st16(rS + 64 * hs + 16 * c, dd);  // over this half's S(x), already read
+                // over this half's dP(x) columns 16c.., read in chunk 0
+                if (depth_item) ptx::tmem_st16(rP + 64 * hs + 16 * c, dl);
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
@@ -753,18 +814,29 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
             ok = false;
         }
         ptx::tc_fence_after();
+        // delta of the whole row = the two column halves' sums (every
+        // compute thread reaches this barrier, whether or not ok)
+        sDelta[hs * 128 + r] = delta;
+        asm volatile("bar.sync 1, %0;" ::"n"(kComputeThreads) : "memory");
+        delta = sDelta[r] + sDelta[128 + r];
         if (ok) {
+            if (row_ok && hs == 0) p.rowD[((long long)b * p.Hq + h) * p.T + t] = Drow + delta;
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.dq) + (((long long)b * p.T + (row_ok ? t : 0)) * p.Hq + h) * kD;
+            const float nds = -delta;
 #pragma unroll 1
             for (int c = 0; c < 2; ++c) {
                 const int col = 64 * hs + 32 * c;  // feature columns of the chunk
-                uint32_t o[32];
+                uint32_t o[32], bq[32];
                 ptx::tmem_ld32(tmem + lane_off + 256 + col, o);
+                ptx::tmem_ld32(tmem + lane_off + 384 + col, bq);
                 ptx::tmem_wait_ld();
                 uint32_t w[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    w[e] = ptx::pack_bf16x2(__uint_as_float(o[2 * e]) * p.scale, __uint_as_float(o[2 * e + 1]) * p.scale);
+                for (int e = 0; e < 16; ++e) {
+                    const float g0 = fmaf(nds, __uint_as_float(bq[2 * e]), __uint_as_float(o[2 * e]));
+                    const float g1 = fmaf(nds, __uint_as_float(bq[2 * e + 1]), __uint_as_float(o[2 * e + 1]));
+                    w[e] = ptx::pack_bf16x2(g0 * p.scale, g1 * p.scale);
+                }
                 if (row_ok) {
                     uint4* d4 = reinterpret_cast<uint4*>(dst + col);
 #pragma unroll
@@ -852,6 +924,24 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s) {
     }
     const int sms = sm_count();
 
+    // ---- dq (first: it turns rowD into the exact D the dK/dV kernels read)
+    DqParams pq;
+    memset(&pq, 0, sizeof(pq));
+    pq.tm_q = tm_q; pq.tm_do = tm_do; pq.tm_k = tm_k; pq.tm_v = tm_v; pq.tm_kd = tm_kd; pq.tm_vd = tm_vd;
+    pq.lse = f.lse; pq.rowD = a.rowD; pq.dq = a.dq;
+    pq.B = f.B; pq.T = f.T; pq.Hq = f.Hq; pq.Hkv = f.Hkv; pq.G = G; pq.n = n; pq.Ld = f.Ld;
+    pq.nqt = (f.T + n - 1) / n;
+    pq.depth_sel = f.depth_sel;
+    pq.sl2 = f.scale * kLog2e; pq.scale = f.scale;
+    pq.status = f.status; pq.wait_limit = f.wait_limit;
+    if ((e = cudaFuncSetAttribute(moda_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem)) !=
+        cudaSuccess)
+        return e;
+    const long long grid_q = (long long)pq.nqt * f.B * f.Hkv;
+    if (grid_q > 0x7fffffffLL) return cudaErrorInvalidValue;
+    moda_bwd_dq_kernel<<<(unsigned)grid_q, kThreads, kDqSmem, s>>>(pq);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
     // ---- dk, dv
     DkvParams pk;
     memset(&pk, 0, sizeof(pk));
@@ -894,24 +984,6 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s) {
         moda_bwd_dkdv_kernel<<<dim3((unsigned)chunks, 1, f.B * f.Hkv), kThreads, kDkvSmem, s>>>(pd);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-
-    // ---- dq
-    DqParams pq;
-    memset(&pq, 0, sizeof(pq));
-    pq.tm_q = tm_q; pq.tm_do = tm_do; pq.tm_k = tm_k; pq.tm_v = tm_v; pq.tm_kd = tm_kd; pq.tm_vd = tm_vd;
-    pq.lse = f.lse; pq.rowD = a.rowD; pq.dq = a.dq;
-    pq.B = f.B; pq.T = f.T; pq.Hq = f.Hq; pq.Hkv = f.Hkv; pq.G = G; pq.n = n; pq.Ld = f.Ld;
-    pq.nqt = (f.T + n - 1) / n;
-    pq.depth_sel = f.depth_sel;
-    pq.sl2 = f.scale * kLog2e; pq.scale = f.scale;
-    pq.status = f.status; pq.wait_limit = f.wait_limit;
-    if ((e = cudaFuncSetAttribute(moda_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem)) !=
-        cudaSuccess)
-        return e;
-    const long long grid_q = (long long)pq.nqt * f.B * f.Hkv;
-    if (grid_q > 0x7fffffffLL) return cudaErrorInvalidValue;
-    moda_bwd_dq_kernel<<<(unsigned)grid_q, kThreads, kDqSmem, s>>>(pq);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     // ---- dk, dv to bf16
     const long long n4 = (long long)f.B * f.T * f.Hkv * kD / 4;

@@ -46,7 +46,8 @@ struct BwdArgs {
     void* dv;
     void* dkd;
     void* dvd;
-    float* rowD;            // [B, Hq, T] fp32 workspace: <dout, out>
+    float* rowD;            // [B, Hq, T] fp32 workspace: <dout, out>, then the
+                            // dq kernel's exact D = sum_j P_j dP_j
     float* dk_acc;          // [B, T, Hkv, d] fp32 workspace (tensor-core path only)
     float* dv_acc;          // [B, T, Hkv, d] fp32 workspace (tensor-core path only)
 };

@@ -14,9 +14,9 @@
 // exits. Larger problems are rejected (MODA_ERR_WORKSPACE) rather than
 // allocated for.
 #include <cstring>
-#include <mutex>
 
 #include "moda_internal.h"
+#include "symbol_addr.h"
 
 namespace moda {
 namespace {
@@ -24,29 +24,11 @@ namespace {
 // The scratch: fp32 row statistics D = rowsum(dout * out), [B, Hq, T].
 __device__ __align__(256) unsigned char g_bwd_noalloc_scratch[MODA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-void* g_scratch_dev_addr[kMaxDevices];
-std::mutex g_scratch_mu;
-
 // In host code `g_bwd_noalloc_scratch` names a host-side stand-in, not the
 // device array: a kernel given it would fault or silently touch the wrong
-// memory. Its device address is resolved once per device, with that device
-// current, and cached.
-cudaError_t scratch_device_addr(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_dev_addr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_bwd_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_dev_addr[dev] = p;
-    }
-    *out = g_scratch_dev_addr[dev];
-    return cudaSuccess;
-}
+// memory. Its device address is resolved with the device current, once per
+// device and context (again after a cudaDeviceReset), and cached.
+SymbolAddr g_scratch_addr(g_bwd_noalloc_scratch);
 
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -76,7 +58,7 @@ extern "C" moda_status moda_bwd_noalloc(const void* q, const void* k, const void
     if (need > MODA_NOALLOC_SCRATCH_BYTES) return MODA_ERR_WORKSPACE;
 
     void* scratch = nullptr;
-    if (scratch_device_addr(&scratch) != cudaSuccess) return MODA_ERR_CUDA;
+    if (g_scratch_addr.get(&scratch) != cudaSuccess) return MODA_ERR_CUDA;
 
     BwdArgs a;
     memset(&a, 0, sizeof(a));

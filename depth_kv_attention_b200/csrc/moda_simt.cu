@@ -241,6 +241,11 @@ __global__ void bwd_rowdot_kernel(BwdArgs a) {
 }
 
 // dq for every query row: causal keys and same-token depth keys.
+// The row statistic D = sum_j P_j dP_j: rowD holds the estimate
+// D~ = <dout, out> on entry (out as the forward stored it); the row's pass
+// over all its keys accumulates delta = sum_j P_j (dP_j - D~) (= D - D~, as
+// sum_j P_j = 1) and bq = sum_j P_j k_j, writes dq = scale (sum_j P_j (dP_j -
+// D~) k_j - delta bq) and stores D = D~ + delta for the dK/dV kernels.
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_dq_simt_kernel(BwdArgs a, int n_tok, int hpc) {
     constexpr int TPR = 4;
@@ -258,15 +263,19 @@ __global__ void __launch_bounds__(256) bwd_dq_simt_kernel(BwdArgs a, int n_tok, 
     const int tc = min(t, f.T - 1), gc = min(g, f.G - 1);
     const int h = kvh * f.G + gc;
 
-    float2 q[S::NP], dO[S::NP], dq[S::NP];
+    float2 q[S::NP], dO[S::NP], dq[S::NP], bq[S::NP];
     load_row<TPR>(static_cast<const T*>(f.q) + b * f.sq.sb + tc * f.sq.st + h * f.sq.sh, f.d, u, q,
                   f.scale * kLog2e);
     load_row<TPR>(static_cast<const T*>(a.dout) + b * f.so.sb + tc * f.so.st + h * f.so.sh, f.d, u, dO);
 #pragma unroll
-    for (int i = 0; i < S::NP; ++i) dq[i] = make_float2(0.f, 0.f);
+    for (int i = 0; i < S::NP; ++i) {
+        dq[i] = make_float2(0.f, 0.f);
+        bq[i] = make_float2(0.f, 0.f);
+    }
     const long long rix = ((long long)b * f.Hq + h) * f.T + tc;
     const float lse2 = f.lse[rix] * kLog2e;
     const float Drow = a.rowD[rix];
+    float delta = 0.f;
 
     // Depth part: dq += dS'_i kd_i over the selected slots (skipped only
     // after the warp-wide shuffles of group_sum, as in the forward).
@@ -280,7 +289,10 @@ __global__ void __launch_bounds__(256) bwd_dq_simt_kernel(BwdArgs a, int n_tok, 
         const float dp = group_sum<TPR>(dot_regs<TPR>(dO, vr));
         if (f.depth_sel && !((sel >> i) & 1ull)) continue;
         const float p = exp2f(s - lse2);
-        axpy_regs<TPR>(dq, p * (dp - Drow), kr);
+        const float ds = p * (dp - Drow);
+        delta += ds;
+        axpy_regs<TPR>(dq, ds, kr);
+        axpy_regs<TPR>(bq, p, kr);
     }
     const int t_last = min(f.T, t0 + n_tok) - 1;
     const T* Kb = static_cast<const T*>(f.k) + b * f.skv.sb + kvh * f.skv.sh;
@@ -294,11 +306,24 @@ __global__ void __launch_bounds__(256) bwd_dq_simt_kernel(BwdArgs a, int n_tok, 
         for (int jj = 0; jj < n; ++jj) {
             const float s = group_sum<TPR>(dot_smem<TPR>(q, sK + jj * kDMax, u));
             const float dp = group_sum<TPR>(dot_smem<TPR>(dO, sV + jj * kDMax, u));
-            if (j0 + jj <= t) axpy_smem<TPR>(dq, exp2f(s - lse2) * (dp - Drow), sK + jj * kDMax, u);
+            if (j0 + jj <= t) {
+                const float p = exp2f(s - lse2);
+                const float ds = p * (dp - Drow);
+                delta += ds;
+                axpy_smem<TPR>(dq, ds, sK + jj * kDMax, u);
+                axpy_smem<TPR>(bq, p, sK + jj * kDMax, u);
+            }
         }
     }
-    if (valid)
+#pragma unroll
+    for (int i = 0; i < S::NP; ++i) {
+        dq[i].x = fmaf(-delta, bq[i].x, dq[i].x);
+        dq[i].y = fmaf(-delta, bq[i].y, dq[i].y);
+    }
+    if (valid) {
         store_row<TPR>(static_cast<T*>(a.dq) + b * f.sq.sb + t * f.sq.st + h * f.sq.sh, f.d, u, dq, f.scale);
+        if (u == 0) a.rowD[rix] = Drow + delta;
+    }
 }
 
 // dk, dv for every sequence key j: rows t >= j of the G heads of its group.

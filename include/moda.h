@@ -145,10 +145,15 @@ size_t moda_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int Ld,
 /*
  * moda_bwd — gradients of moda_fwd for upstream gradient dout. The pages give
  * no backward pass; this is the derivative of the forward definition above:
- *   P = exp(s - lse), D = <dout, out>, dS = P * (dP - D) with
- *   dP = [dout.v_j || dout.vd_i];  dq = scale*(sum_j dS_j k_j + sum_i dS'_i kd_i),
+ *   P = exp(s - lse), dP = [dout.v_j || dout.vd_i], D = sum P dP (over the
+ *   row's sequence and depth keys), dS = P * (dP - D);
+ *   dq = scale*(sum_j dS_j k_j + sum_i dS'_i kd_i),
  *   dk_j = scale*sum dS_j q, dv_j = sum P_j dout (over rows t >= j of the
  *   group's G heads), dkd / dvd likewise over the G heads of the same token.
+ * D equals <dout, out> of the exact output. The library takes <dout, out>
+ * of the output it is given only as a first estimate and corrects it from
+ * its own recomputed P and dP, so the gradients do not inherit the rounding
+ * of the stored (bf16) output, which wide depth keys would amplify.
  *   q,k,v,kd,vd,out   in   as in moda_fwd (out is moda_fwd's output)
  *   lse               in   moda_fwd's lse
  *   dout [B,T,Hq,d]   in   upstream gradient
@@ -212,7 +217,10 @@ moda_status moda_bwd_sel(const void* q, const void* k, const void* v,
  *     return MODA_ERR_WORKSPACE with nothing launched.
  *   - Set-up: the first call on each device resolves the array's device
  *     address (cudaGetSymbolAddress, with that device current). Make that
- *     first call before any stream capture on the device.
+ *     first call before any stream capture on the device. The address is
+ *     kept per CUDA context: after cudaDeviceReset (or a new primary
+ *     context) the next call resolves it again, so make that call outside
+ *     a capture too.
  *   - Sharing: every call on a device uses the same array, which keeps the
  *     previous call's contents (nothing needs clearing: the backward writes
  *     every entry before reading it). Calls whose kernels overlap on the GPU
@@ -268,6 +276,35 @@ moda_status moda_fwd_packed(const void* q, const void* k, const void* v,
                             int B, int T, int Hq, int Hkv, int d, int Ld,
                             moda_dtype dtype, float scale,
                             void* out, float* lse, void* stream);
+
+/*
+ * moda_fwd_host — moda_fwd end to end from HOST buffers: enqueues on
+ * `stream` the host-to-device copies of q, k, v, kd, vd into the caller's
+ * device staging buffer, the forward on the staged inputs, and the
+ * device-to-host copies of out and lse. No pages describe this; it is the
+ * boundary a host program without device buffers of its own uses.
+ *   q, k, v, kd, vd   in   HOST pointers, layouts as in moda_fwd (kd / vd NULL
+ *                          iff Ld == 0)
+ *   out, lse          out  HOST pointers (lse may be NULL)
+ *   staging           in   DEVICE buffer of >= moda_fwd_host_staging_bytes(...)
+ *                          bytes, 256-byte aligned; contents on entry ignored,
+ *                          holds the staged tensors afterwards
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister) for
+ * the copies to be asynchronous; with pageable memory the copies still work
+ * but block the calling thread. Returns once everything is enqueued; out and
+ * lse hold the results when the stream reaches the end of the call (e.g.
+ * after moda_device_status(stream)). Errors: as moda_fwd, MODA_ERR_WORKSPACE
+ * for a missing or short staging buffer, MODA_ERR_CUDA if a copy cannot be
+ * enqueued.
+ */
+size_t moda_fwd_host_staging_bytes(int B, int T, int Hq, int Hkv, int d, int Ld,
+                                   moda_dtype dtype);
+moda_status moda_fwd_host(const void* q, const void* k, const void* v,
+                          const void* kd, const void* vd,
+                          int B, int T, int Hq, int Hkv, int d, int Ld,
+                          moda_dtype dtype, float scale,
+                          void* out, float* lse,
+                          void* staging, size_t staging_bytes, void* stream);
 
 /*
  * moda_device_status — synchronises `stream`, then reads and clears the

@@ -44,6 +44,11 @@ def compare(name, got, want, dtype, what="out", grad=False):
     if grad and dtype == "bf16":
         allowed = tol["max_abs"] + np.abs(want) * 2.0 ** -8
         worst = float((err / allowed).max()) if err.size else 0.0
+        # how many elements needed the relative term (error above the plain
+        # stated bound), reported with every gradient comparison
+        n_rel = int(np.count_nonzero(err > tol["max_abs"]))
+        print(f"{name}: {n_rel} of {err.size} elements above {tol['max_abs']} "
+              f"(within 2^-8 |g| of it), max-abs {mx:.3e}")
         assert worst <= 1.0, f"{name}: max-abs {mx:.3e}, {worst:.2f}x the bf16-scaled bound"
     else:
         assert mx <= tol["max_abs"], f"{name}: max-abs {mx:.3e} > {tol['max_abs']}"

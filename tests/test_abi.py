@@ -122,3 +122,26 @@ def test_depth_write_validation():
     assert depth_write(k=None) == 1
     assert depth_write(kd=P + 8) == 3
     assert depth_write(d=12) == 2          # 24 bytes per bf16 row
+
+
+def fwd_host(staging=P, staging_bytes=1 << 30, q=P, B=1, T=8, Hq=4, Hkv=2, d=64, Ld=2, dt=0):
+    return moda._c_fwd_host(q, P, P, P, P, B, T, Hq, Hkv, d, Ld, dt, 0.125, P, P, staging,
+                            staging_bytes, None)
+
+
+def test_fwd_host_staging_size_and_validation():
+    """moda_fwd_host stages q, k, v, kd, vd, out and lse at 256-byte-aligned
+    offsets of the caller's device buffer; a missing, short or misaligned
+    staging buffer and bad shapes are rejected before any copy."""
+    B, T, Hq, Hkv, d, Ld = 1, 8, 4, 2, 64, 2
+    r = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    want = (2 * r(B * T * Hq * d * 2) + 2 * r(B * T * Hkv * d * 2) + 2 * r(B * T * Ld * Hkv * d * 2)
+            + r(B * Hq * T * 4))
+    assert moda._c_host_bytes(B, T, Hq, Hkv, d, Ld, 0) == want
+    assert moda._c_host_bytes(B, T, 3, Hkv, d, Ld, 0) == 0
+    assert fwd_host(staging=None) == 4
+    assert fwd_host(staging_bytes=want - 1) == 4
+    assert fwd_host(staging=P + 16) == 3
+    assert fwd_host(q=None) == 1
+    assert fwd_host(Hq=3) == 1
+    assert fwd_host(d=256) == 2

@@ -55,3 +55,43 @@ def test_reference_arm_runs_on_rank0_only(monkeypatch):
     class A:
         steps, warmup, ref_rows = 1, 3, 4
     assert bench.reference_arm(A, bench.WORKLOADS["tiny_f32"]) == 0
+
+
+def test_launcher_starts_two_ranks_and_partitions_heads():
+    """``python bench.py --gpus 2`` outside torchrun starts the two ranks
+    itself (torch.distributed.run, gloo in the dry run); the kv-head shards
+    of the ranks are disjoint, cover every head and add up to the whole
+    workload's FLOPs (strong scaling)."""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dry-run",
+                        "--partition", "heads", "--workload", "t4k"],
+                       capture_output=True, text=True, timeout=240, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][-1])
+    assert line["n_gpus"] == 2 and line["scaling"] == "strong"
+    shares = sorted(line["shares"], key=lambda s: s["rank"])
+    assert [s["kv_heads"] for s in shares] == [[0, 2], [2, 4]]
+    assert [s["q_heads"] for s in shares] == [[0, 16], [16, 32]]
+    assert line["job_flops"] == line["full_flops"]
+
+
+def test_head_shards_need_no_exchange():
+    """The oracle's output for each rank's kv-head shard, computed from that
+    shard's inputs alone, equals the full workload's output on those heads:
+    the head partition needs no data exchange between ranks."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle
+    from moda_inputs import Workload, make_inputs
+    w = Workload("shard", 2, 40, 8, 4, 16, 3, "f32", 77)
+    x = make_inputs(w)
+    full, full_lse = oracle.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], w.scale)
+    for world in (2, 4):
+        for rank in range(world):
+            ws, xs = bench.shard_heads(w, x, rank, world)
+            o, l = oracle.forward(xs["q"], xs["k"], xs["v"], xs["kd"], xs["vd"], ws.scale)
+            q0 = rank * (w.Hq // world)
+            np.testing.assert_array_equal(o, full[:, :, q0:q0 + ws.Hq])
+            np.testing.assert_array_equal(l, full_lse[:, q0:q0 + ws.Hq])

@@ -93,15 +93,16 @@ def check_sampled(w, impl, heads=None, x=None, n_rows=256):
 
 @pytest.mark.parametrize("impl", ["tc", "simt"])
 def test_t16k_b2_sampled_with_depth_difference(impl):
-    """2x16K, Ld=24 and Ld=0 on sampled rows; the lse difference
-    lse(Ld) - lse(0) (the depth keys' contribution) matches the oracle's."""
+    """2x16K, Ld=24 and Ld=0 on 256 sampled rows of every head (the SIMT
+    kernels on 4 heads); the lse difference lse(Ld) - lse(0) (the depth keys'
+    contribution) matches the oracle's."""
     w = WORKLOADS["t16k_b2"]
-    heads = [0, 7, 13, 31]
+    heads = list(range(w.Hq)) if impl == "tc" else [0, 7, 13, 31]
     x = make_inputs(w)
-    r24 = check_sampled(w, impl, heads, x, n_rows=96)
+    r24 = check_sampled(w, impl, heads, x, n_rows=256)
     w0 = w.with_(Ld=0)
     x0 = dict(x, kd=x["kd"][:, :, :0].contiguous(), vd=x["vd"][:, :, :0].contiguous())
-    r0 = check_sampled(w0, impl, heads, x0, n_rows=96)
+    r0 = check_sampled(w0, impl, heads, x0, n_rows=256)
     for key in r24:
         got = r24[key][0] - r0[key][0]
         want = r24[key][1] - r0[key][1]
@@ -128,3 +129,18 @@ def test_packed_depth_matches_native():
     ro, rl = oracle.forward(*(x[n].cpu() for n in ("q", "k", "v", "kd", "vd")), w.scale)
     compare("packed out", f64(o2), ro, "bf16")
     compare("packed lse", f64(l2), rl, "bf16", what="lse")
+
+
+def test_fwd_host_entry_matches_device_forward():
+    """moda_fwd_host (host buffers in and out, device staging) gives the
+    device-pointer forward's output bit for bit, and the oracle's."""
+    w = Workload("host", 2, 333, 16, 2, 128, 5, "bf16", 22)
+    x = make_inputs(w)
+    pinned = {k: v.pin_memory() for k, v in x.items()}
+    out_h, lse_h = moda.moda_fwd_from_host(pinned["q"], pinned["k"], pinned["v"], pinned["kd"],
+                                           pinned["vd"], w.scale)
+    out, lse = run_fwd(w, x, "auto")
+    assert torch.equal(out_h, out.cpu()) and torch.equal(lse_h, lse.cpu())
+    ro, rl = oracle.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], w.scale)
+    compare("host out", f64(out_h), ro, "bf16")
+    compare("host lse", f64(lse_h), rl, "bf16", what="lse")

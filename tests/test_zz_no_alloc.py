@@ -44,6 +44,22 @@ def test_noalloc_backward_matches_moda_bwd_on_two_calls_in_a_row():
             assert torch.equal(g, s), f"{w.name} {n}: differs from moda_bwd_ex on the same kernels"
 
 
+def test_noalloc_fp32_matches_scalar_backward_and_oracle():
+    """fp32 inputs (the tiny fp32 workload's shape: T=128, G=4, d=64, Ld=4):
+    the float row statistics in the shared array and the fp32 kernels, bit
+    for bit against moda_bwd on the same kernels and within 1e-5 of the
+    float64 oracle's exact derivative, on two calls in a row."""
+    import oracle
+    w = Workload("noalloc_f32", 1, 128, 4, 1, 64, 4, "f32", 63)
+    x = make_inputs(w, with_dout=True)
+    want = oracle.backward(x["q"], x["k"], x["v"], x["kd"], x["vd"], x["dout"], w.scale)
+    for _ in range(2):
+        ref, same, got = _grads(w)
+        for n, s, g, r in zip(NAMES, same, got, want):
+            assert torch.equal(g, s), f"{w.name} {n}: differs from moda_bwd_ex on the same kernels"
+            compare(f"{w.name} {n} vs oracle", f64(g), r, "f32")
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch():
     limit = 16 * 1024 * 1024
     B, T, Hq = 1, limit // (4 * 32) + 1, 32  # B*Hq*T*4 bytes just over the array
