@@ -54,7 +54,8 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["to_f64", "forward", "forward_rows", "backward", "depth_write"]
+__all__ = ["to_f64", "forward", "forward_rows", "backward", "depth_write", "quantize_q8",
+           "dequantize_q8", "depth_write_q8"]
 
 
 def to_f64(x) -> np.ndarray:
@@ -227,3 +228,56 @@ def depth_write(kd, vd, k, v, slot: int):
     kd2[:, :, slot] = np.asarray(k)
     vd2[:, :, slot] = np.asarray(v)
     return kd2, vd2
+
+
+# ------------------------------------------------------------ 8-bit depth KV
+#
+# "动态混合深度注意力机制MoDA技术解析" (mhpn.cn) §4.2 (memory tips): where device
+# memory is short, the depth KV of models beyond 32 layers can be stored with
+# 8-bit quantisation. The page names no format. Reading used here: symmetric
+# per-row absmax int8, one float32 scale per (b, t, slot, kv-head) row of d
+# values:
+#
+#   amax   = max_c |x_c|                     (x: the row in float32)
+#   sigma  = fl32(amax / 127)                (0 for an all-zero row)
+#   code_c = clamp(round_half_even(fl32(x_c / sigma)), -127, 127)
+#   x^_c   = sigma * code_c                  (the value the method attends to)
+#
+# fl32 is one IEEE float32 operation, rounded to nearest even: both sides of
+# a comparison take every decision that fixes a code in float32. The
+# attention itself is the unchanged MoDA read step over the dequantised depth
+# keys and values x^.
+
+
+def quantize_q8(x):
+    """Symmetric per-row int8 quantisation of the last axis of ``x`` (a float
+    array or tensor; bf16 is upcast exactly). Returns (codes int8 [..., d],
+    scales float32 [...])."""
+    xf = np.asarray(to_f64(x), dtype=np.float64).astype(np.float32)  # exact for bf16 / f32 inputs
+    amax = np.max(np.abs(xf), axis=-1)
+    sigma = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(sigma > 0, sigma, np.float32(1.0)).astype(np.float32)
+    r = (xf / safe[..., None]).astype(np.float32)
+    codes = np.clip(np.rint(r), -127, 127)                       # rint: ties to even
+    codes = np.where(sigma[..., None] > 0, codes, 0).astype(np.int8)
+    return codes, sigma
+
+
+def dequantize_q8(codes, scales):
+    """x^ = scale * code, exactly, as float64 [..., d]."""
+    return np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[..., None]
+
+
+def depth_write_q8(kd8, vd8, kd_scale, vd_scale, k, v, slot: int):
+    """The write step into an 8-bit depth cache: k, v [B,T,Hkv,d] quantised
+    row by row (``quantize_q8``) into slot ``slot`` of the codes kd8, vd8
+    [B,T,Ld,Hkv,d] and scales kd_scale, vd_scale [B,T,Ld,Hkv]. Returns new
+    arrays (kd8', vd8', kd_scale', vd_scale'); other slots unchanged."""
+    out = [np.array(a, copy=True) for a in (kd8, vd8, kd_scale, vd_scale)]
+    ck, sk = quantize_q8(k)
+    cv, sv = quantize_q8(v)
+    out[0][:, :, slot] = ck
+    out[1][:, :, slot] = cv
+    out[2][:, :, slot] = sk
+    out[3][:, :, slot] = sv
+    return tuple(out)

@@ -460,3 +460,102 @@ def test_depth_write_against_loops_and_forward():
     o2, l2 = brute_force(q, ks, vs, stacked_k, stacked_v, 0.5)
     np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-12)
     np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------ 8-bit depth KV
+def test_q8_hand_worked_rows_and_ties():
+    """Rows whose scale is exact (amax 127 -> sigma 1, amax 254 -> sigma 2):
+    the codes are the nearest integers of x / sigma with ties to even, the
+    amax element maps to +-127, an all-zero row has scale 0 and codes 0."""
+    rows = np.array([[127.0, 2.5, 3.5, -2.5, -3.5, 0.5, 1.5, -127.0],
+                     [254.0, 5.0, 7.0, -5.0, 1.0, 3.0, -254.0, 0.0],
+                     [0.0] * 8], dtype=np.float32)
+    codes, sigma = om.quantize_q8(rows)
+    assert sigma.tolist() == [1.0, 2.0, 0.0]
+    assert codes.tolist() == [[127, 2, 4, -2, -4, 0, 2, -127],
+                              [127, 2, 4, -2, 0, 2, -127, 0],
+                              [0] * 8]
+    assert codes.dtype == np.int8 and sigma.dtype == np.float32
+
+
+def test_q8_nearest_code_and_error_bound():
+    """On random bf16 rows: every code is the nearest multiple of sigma (no
+    neighbour code is closer), |x - sigma*code| <= sigma/2 up to the float32
+    rounding of x / sigma, codes lie in [-127, 127], and each row's largest
+    |x| maps to |code| = 127."""
+    g = torch.Generator("cpu")
+    g.manual_seed(5)
+    x = (torch.randn(64, 7, 128, generator=g) * torch.rand(64, 7, 1, generator=g) * 10).to(torch.bfloat16)
+    xf = om.to_f64(x)
+    codes, sigma = om.quantize_q8(x)
+    c = codes.astype(np.float64)
+    s = sigma.astype(np.float64)[..., None]
+    err = np.abs(xf - s * c)
+    assert np.all(np.abs(c) <= 127)
+    # x / sigma is rounded to float32 before the integer rounding: half an
+    # ulp of a quotient below 128 is at most 2^-18, so a code may sit up to
+    # sigma * 2^-18 beyond the exact half-way point
+    assert np.all(err <= s * (0.5 + 2.0 ** -17) + 1e-30)
+    for dc in (-1, 1):
+        nb = np.clip(c + dc, -127, 127)
+        assert np.all(err <= np.abs(xf - s * nb) + s * 2.0 ** -16)
+    amax_idx = np.argmax(np.abs(xf), axis=-1)[..., None]
+    assert np.all(np.abs(np.take_along_axis(c, amax_idx, -1)) == 127)
+    # the scale is amax / 127 in float32
+    np.testing.assert_array_equal(sigma, (np.max(np.abs(xf), -1).astype(np.float32) / np.float32(127)))
+
+
+def test_q8_dequantise_is_exact_and_write_step_touches_one_slot():
+    g = torch.Generator("cpu")
+    g.manual_seed(6)
+    B, T, Ld, Hkv, d = 2, 5, 3, 2, 16
+    kd = torch.randn(B, T, Ld, Hkv, d, generator=g).to(torch.bfloat16)
+    vd = torch.randn(B, T, Ld, Hkv, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, T, Hkv, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, T, Hkv, d, generator=g).to(torch.bfloat16)
+    ck, sk = om.quantize_q8(kd)
+    cv, sv = om.quantize_q8(vd)
+    deq = om.dequantize_q8(ck, sk)
+    for idx in [(0, 0, 0, 0, 3), (1, 4, 2, 1, 15), (1, 2, 1, 0, 0)]:
+        assert deq[idx] == float(ck[idx]) * float(sk[idx[:-1]])  # one exact product
+    kd8, vd8, sk2, sv2 = om.depth_write_q8(ck, cv, sk, sv, k, v, 1)
+    for slot in (0, 2):
+        np.testing.assert_array_equal(kd8[:, :, slot], ck[:, :, slot])
+        np.testing.assert_array_equal(sv2[:, :, slot], sv[:, :, slot])
+    c1, s1 = om.quantize_q8(k)
+    np.testing.assert_array_equal(kd8[:, :, 1], c1)
+    np.testing.assert_array_equal(sk2[:, :, 1], s1)
+    c2, s2 = om.quantize_q8(v)
+    np.testing.assert_array_equal(vd8[:, :, 1], c2)
+    np.testing.assert_array_equal(sv2[:, :, 1], s2)
+
+
+def test_planted_q8_mistakes_are_caught(monkeypatch):
+    """Truncation instead of rounding, ties away from zero, and a scale of
+    amax / 128 each fail the hand-worked or the nearest-code pin."""
+    real = om.quantize_q8
+
+    def trunc(x):
+        xf = np.asarray(om.to_f64(x)).astype(np.float32)
+        sigma = (np.max(np.abs(xf), -1) / np.float32(127)).astype(np.float32)
+        safe = np.where(sigma > 0, sigma, 1).astype(np.float32)
+        return np.trunc(xf / safe[..., None]).astype(np.int8), sigma
+
+    def away(x):
+        xf = np.asarray(om.to_f64(x)).astype(np.float32)
+        sigma = (np.max(np.abs(xf), -1) / np.float32(127)).astype(np.float32)
+        safe = np.where(sigma > 0, sigma, 1).astype(np.float32)
+        r = xf / safe[..., None]
+        return (np.sign(r) * np.floor(np.abs(r) + 0.5)).astype(np.int8), sigma
+
+    def scale128(x):
+        xf = np.asarray(om.to_f64(x)).astype(np.float32)
+        sigma = (np.max(np.abs(xf), -1) / np.float32(128)).astype(np.float32)
+        safe = np.where(sigma > 0, sigma, 1).astype(np.float32)
+        return np.clip(np.rint(xf / safe[..., None]), -127, 127).astype(np.int8), sigma
+
+    for bad in (trunc, away, scale128):
+        monkeypatch.setattr(om, "quantize_q8", bad)
+        with pytest.raises(AssertionError):
+            test_q8_hand_worked_rows_and_ties()
+        monkeypatch.setattr(om, "quantize_q8", real)
