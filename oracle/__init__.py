@@ -5,4 +5,4 @@ and reference arm may import this package. It shares no code with the CUDA
 path and imports nothing from it.
 """
 from .moda_oracle import (backward, depth_write, depth_write_q8, dequantize_q8, forward,  # noqa: F401
-                          forward_rows, quantize_q8, to_f64)
+                          forward_rows, quantize_q8, round_to_bf16, to_f64)

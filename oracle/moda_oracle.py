@@ -55,7 +55,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = ["to_f64", "forward", "forward_rows", "backward", "depth_write", "quantize_q8",
-           "dequantize_q8", "depth_write_q8"]
+           "dequantize_q8", "depth_write_q8", "round_to_bf16"]
 
 
 def to_f64(x) -> np.ndarray:
@@ -241,12 +241,15 @@ def depth_write(kd, vd, k, v, slot: int):
 #   amax   = max_c |x_c|                     (x: the row in float32)
 #   sigma  = fl32(amax / 127)                (0 for an all-zero row)
 #   code_c = clamp(round_half_even(fl32(x_c / sigma)), -127, 127)
-#   x^_c   = sigma * code_c                  (the value the method attends to)
+#   x^_c   = the cache's storage dtype of fl32(sigma * code_c)
+#            (bf16, round to nearest even, for a bf16 cache; float32 itself
+#             for a float32 cache): the 8-bit cache decompresses into the
+#             same type the unquantised depth cache holds
 #
 # fl32 is one IEEE float32 operation, rounded to nearest even: both sides of
-# a comparison take every decision that fixes a code in float32. The
-# attention itself is the unchanged MoDA read step over the dequantised depth
-# keys and values x^.
+# a comparison take every decision that fixes a code or a value in float32.
+# The attention itself is the unchanged MoDA read step over the dequantised
+# depth keys and values x^.
 
 
 def quantize_q8(x):
@@ -263,9 +266,25 @@ def quantize_q8(x):
     return codes, sigma
 
 
-def dequantize_q8(codes, scales):
-    """x^ = scale * code, exactly, as float64 [..., d]."""
-    return np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[..., None]
+def round_to_bf16(x32):
+    """float32 -> the nearest bf16 value (ties to even mantissa), returned as
+    float32: keep the upper 16 bits of the float32 pattern after adding half
+    of the dropped range plus the parity of the kept bit (finite inputs)."""
+    b = np.asarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000
+    return b.astype(np.uint32).view(np.float32)
+
+
+def dequantize_q8(codes, scales, dtype: str = "bf16"):
+    """x^ = fl32(scale * code) in the cache's storage dtype ("bf16" or
+    "f32"), returned exactly as float64 [..., d]."""
+    prod = (np.asarray(codes, dtype=np.float32)
+            * np.asarray(scales, dtype=np.float32)[..., None]).astype(np.float32)
+    if dtype == "bf16":
+        prod = round_to_bf16(prod)
+    elif dtype != "f32":
+        raise ValueError(dtype)
+    return prod.astype(np.float64)
 
 
 def depth_write_q8(kd8, vd8, kd_scale, vd_scale, k, v, slot: int):

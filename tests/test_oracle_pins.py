@@ -515,9 +515,17 @@ def test_q8_dequantise_is_exact_and_write_step_touches_one_slot():
     v = torch.randn(B, T, Hkv, d, generator=g).to(torch.bfloat16)
     ck, sk = om.quantize_q8(kd)
     cv, sv = om.quantize_q8(vd)
-    deq = om.dequantize_q8(ck, sk)
+    # float32 cache: one float32 product; bf16 cache: that product rounded to
+    # bf16 exactly as torch rounds float32 to bfloat16 (a library routine)
+    deq32 = om.dequantize_q8(ck, sk, "f32")
+    deq16 = om.dequantize_q8(ck, sk, "bf16")
     for idx in [(0, 0, 0, 0, 3), (1, 4, 2, 1, 15), (1, 2, 1, 0, 0)]:
-        assert deq[idx] == float(ck[idx]) * float(sk[idx[:-1]])  # one exact product
+        assert deq32[idx] == float(np.float32(ck[idx]) * np.float32(sk[idx[:-1]]))
+    prod = torch.from_numpy(deq32.astype(np.float32))
+    np.testing.assert_array_equal(deq16, prod.to(torch.bfloat16).to(torch.float64).numpy())
+    # ties: 1 + 2^-8 lies half-way between bf16 neighbours 1 and 1 + 2^-7
+    ties = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8), 3.0], dtype=np.float32)
+    assert om.round_to_bf16(ties).tolist() == [1.0, 1 + 2.0 ** -6, -1.0, 3.0]
     kd8, vd8, sk2, sv2 = om.depth_write_q8(ck, cv, sk, sv, k, v, 1)
     for slot in (0, 2):
         np.testing.assert_array_equal(kd8[:, :, slot], ck[:, :, slot])
