@@ -333,6 +333,8 @@ def measure_secondary(moda, w, world, kernel, steps=20, warmup=3):
            "ld0_fwd_ms": ms0, "overhead_vs_ld0": ms / ms0 - 1.0,
            "depth_stream_gbs": depth_stream_gbs(w, ms, ms0),
            "timing": f"Ld and Ld=0 arms interleaved in blocks of 5, {steps} calls each"}
+    if w.Ld and kernel != "simt":
+        res["depth_q8"] = measure_q8(moda, w, x, world, kernel, step, step0, steps, warmup)
     # Selected depth: each token keeps a window of its most recent slots
     # (width uniform in [0, Ld]), the same FLOPs are issued (whole tiles).
     sel = pack_depth_sel(make_depth_sel(w, "window")).cuda() if w.Ld else None
@@ -353,6 +355,25 @@ def measure_secondary(moda, w, world, kernel, steps=20, warmup=3):
     del x
     torch.cuda.empty_cache()
     return res
+
+
+def measure_q8(moda, w, x, world, kernel, step_bf16, step_ld0, steps, warmup):
+    """The 8-bit depth cache against the bf16 one and Ld = 0: three forwards
+    interleaved. The depth stream shrinks from 2d to d + 4 bytes per row."""
+    kd8, vd8, ks, vs = moda.moda_depth_quantize_q8(x["kd"], x["vd"])
+    out = torch.empty_like(x["q"])
+    lse = torch.empty((w.B, w.Hq, w.T), device="cuda", dtype=torch.float32)
+
+    def step_q8():
+        moda.moda_fwd_q8(x["q"], x["k"], x["v"], kd8, vd8, ks, vs, w.scale, out=out, lse=lse, impl=kernel)
+    msb, msq, ms0 = timed_interleaved([step_bf16, step_q8, step_ld0], steps, warmup, world)
+    q8_bytes = 2 * w.B * w.T * w.Ld * w.Hkv * (w.d + 4)
+    return {"fwd_q8_ms": msq, "fwd_bf16_depth_ms": msb, "ld0_fwd_ms": ms0,
+            "q8_overhead_vs_ld0": msq / ms0 - 1.0, "bf16_overhead_vs_ld0": msb / ms0 - 1.0,
+            "q8_vs_bf16_depth": msq / msb - 1.0,
+            "depth_bytes_q8": q8_bytes, "depth_bytes_bf16": depth_stream_bytes(w),
+            "timing": f"bf16-depth, 8-bit-depth and Ld=0 forwards interleaved in blocks of 5, "
+                      f"{steps} calls each"}
 
 
 def depth_stream_bytes(w) -> int:
@@ -535,6 +556,9 @@ def main():
                                     f"{args.extra_steps} calls each ({ms_a:.3f} vs {ms0:.3f} ms)")
         extra["depth_stream_gbs"] = depth_stream_gbs(w, ms_a, ms0)
         extra["depth_stream_bytes"] = depth_stream_bytes(w)
+        if args.kernel != "simt":
+            extra["depth_q8"] = measure_q8(moda, w, x, world, args.kernel, step, step0, args.extra_steps,
+                                           args.warmup)
         del out0, lse0
         # the optional repack: moda_pack_depth + moda_fwd_packed against the
         # forward on the native depth layout

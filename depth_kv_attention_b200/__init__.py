@@ -22,7 +22,8 @@ __all__ = [
     "moda_fwd", "moda_fwd_sel", "moda_bwd", "moda_bwd_sel", "moda_bwd_workspace_bytes", "moda_bwd_noalloc", "moda_pack_depth",
     "moda_pack_depth_bytes", "moda_fwd_packed", "moda_depth_write", "moda_device_status",
     "moda_debug_set_wait_limit", "moda_debug_exp2_poly", "moda_fwd_from_host",
-    "moda_fwd_host_staging_bytes",
+    "moda_fwd_host_staging_bytes", "moda_fwd_q8", "moda_depth_quantize_q8", "moda_depth_write_q8",
+    "moda_depth_slot_layout", "depth_slot_view",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoda.so")
@@ -64,6 +65,11 @@ _c_wait_limit = _sig("moda_debug_set_wait_limit", _i, [ctypes.c_uint32])
 _c_exp2_poly = _sig("moda_debug_exp2_poly", _i, [_vp, _vp, _i, _vp])
 _c_bwd_noalloc = _sig("moda_bwd_noalloc", _i, [_vp] * 8 + _DIMS + [_i, _f] + [_vp] * 5 + [_vp])
 _c_host_bytes = _sig("moda_fwd_host_staging_bytes", _sz, _DIMS + [_i])
+_c_slot_layout = _sig("moda_depth_slot_layout", _i, [_i] * 6 + [ctypes.POINTER(ctypes.c_longlong),
+                                                                  ctypes.POINTER(ctypes.c_longlong)])
+_c_fwd_q8 = _sig("moda_fwd_q8", _i, [_vp] * 7 + _DIMS + [_i, _f, _vp, _vp, _vp, _i])
+_c_quant_q8 = _sig("moda_depth_quantize_q8", _i, [_vp, _vp] + [_i] * 5 + [_i] + [_vp] * 4 + [_vp])
+_c_write_q8 = _sig("moda_depth_write_q8", _i, [_vp, _vp] + [_i] * 6 + [_i] + [_vp] * 4 + [_vp])
 _c_fwd_host = _sig("moda_fwd_host", _i, [_vp] * 5 + _DIMS + [_i, _f, _vp, _vp, _vp, _sz, _vp])
 
 
@@ -295,6 +301,79 @@ def moda_depth_write(k, v, kd, vd, slot: int, stream=None):
         _check(_c_depth_write(_ptr(k), _ptr(v), B, T, Hkv, d, Ld, slot, _DTYPE[k.dtype], _ptr(kd),
                               _ptr(vd), _stream(stream)), "moda_depth_write")
     return kd, vd
+
+
+def moda_depth_quantize_q8(kd, vd, out=None, stream=None):
+    """8-bit depth cache of kd, vd [B,T,Ld,Hkv,d] (``moda_depth_quantize_q8``).
+    Returns (kd8, vd8, kd_scale, vd_scale): int8 codes [B,T,Ld,Hkv,d] and fp32
+    row scales [B,T,Ld,Hkv]; ``out`` may supply those four tensors."""
+    _check_tensors(kd, vd)
+    B, T, Ld, Hkv, d = kd.shape
+    if out is None:
+        out = (torch.empty(kd.shape, dtype=torch.int8, device=kd.device),
+               torch.empty(kd.shape, dtype=torch.int8, device=kd.device),
+               torch.empty(kd.shape[:-1], dtype=torch.float32, device=kd.device),
+               torch.empty(kd.shape[:-1], dtype=torch.float32, device=kd.device))
+    _check_tensors(*out)
+    with torch.cuda.device(kd.device):
+        _check(_c_quant_q8(_ptr(kd), _ptr(vd), B, T, Hkv, d, Ld, _DTYPE[kd.dtype], *(_ptr(t) for t in out),
+                           _stream(stream)), "moda_depth_quantize_q8")
+    return out
+
+
+def moda_depth_write_q8(k, v, kd8, vd8, kd_scale, vd_scale, slot: int, stream=None):
+    """The write step into an 8-bit depth cache (``moda_depth_write_q8``): k, v
+    [B,T,Hkv,d] quantised into slot ``slot`` of kd8, vd8 and their scales, in
+    place. Returns (kd8, vd8, kd_scale, vd_scale)."""
+    _check_tensors(k, v, kd8, vd8, kd_scale, vd_scale)
+    B, T, Hkv, d = k.shape
+    Ld = kd8.shape[2]
+    if kd8.dtype != torch.int8 or kd_scale.dtype != torch.float32 or tuple(kd8.shape) != (B, T, Ld, Hkv, d):
+        raise ValueError("moda_depth_write_q8: int8 kd8 [B,T,Ld,Hkv,d] and fp32 scales [B,T,Ld,Hkv] expected")
+    with torch.cuda.device(k.device):
+        _check(_c_write_q8(_ptr(k), _ptr(v), B, T, Hkv, d, Ld, slot, _DTYPE[k.dtype], _ptr(kd8), _ptr(vd8),
+                           _ptr(kd_scale), _ptr(vd_scale), _stream(stream)), "moda_depth_write_q8")
+    return kd8, vd8, kd_scale, vd_scale
+
+
+def moda_fwd_q8(q, k, v, kd8, vd8, kd_scale, vd_scale, scale: float | None = None, out=None, lse=None,
+                impl: str = "auto", stream=None):
+    """MoDA forward over an 8-bit depth cache (``moda_fwd_q8``). Returns (out, lse)."""
+    if kd8 is not None and kd8.shape[2] == 0:
+        kd8 = vd8 = kd_scale = vd_scale = None
+    _check_tensors(q, k, v, kd8, vd8, kd_scale, vd_scale, out, lse)
+    B, T, Hq, Hkv, d, Ld = _dims(q, k, kd8)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
+    with torch.cuda.device(q.device):
+        _check(_c_fwd_q8(_ptr(q), _ptr(k), _ptr(v), _ptr(kd8), _ptr(vd8), _ptr(kd_scale), _ptr(vd_scale),
+                         B, T, Hq, Hkv, d, Ld, _DTYPE[q.dtype], scale, _ptr(out), _ptr(lse),
+                         _stream(stream), _IMPL[impl]), "moda_fwd_q8")
+    return out, lse
+
+
+def moda_depth_slot_layout(B, T, Hkv, d, Ld, slot):
+    """(offset, strides) of depth slot ``slot`` inside a native cache
+    [B,T,Ld,Hkv,d], in elements (``moda_depth_slot_layout``)."""
+    off = ctypes.c_longlong()
+    st = (ctypes.c_longlong * 4)()
+    _check(_c_slot_layout(B, T, Hkv, d, Ld, slot, ctypes.byref(off), st), "moda_depth_slot_layout")
+    return off.value, tuple(st)
+
+
+def depth_slot_view(kd, slot: int):
+    """Slot ``slot`` of a depth cache kd [B,T,Ld,Hkv,d] as a strided
+    [B, T, Hkv, d] view (no copy), per ``moda_depth_slot_layout``: a producer
+    that writes its K or V into this view (e.g. a projection GEMM with
+    ``out=view.view(B*T, Hkv*d)``-style leading dimension Ld*Hkv*d) fills the
+    cache in place."""
+    B, T, Ld, Hkv, d = kd.shape
+    off, st = moda_depth_slot_layout(B, T, Hkv, d, Ld, slot)
+    return kd.as_strided((B, T, Hkv, d), st, kd.storage_offset() + off)
 
 
 def moda_device_status(stream=None) -> int:

@@ -271,6 +271,84 @@ moda_status moda_depth_write(const void* k, const void* v, int B, int T, int Hkv
     return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
 }
 
+moda_status moda_fwd_q8(const void* q, const void* k, const void* v, const int8_t* kd8, const int8_t* vd8,
+                        const float* kd_scale, const float* vd_scale, int B, int T, int Hq, int Hkv, int d,
+                        int Ld, moda_dtype dtype, float scale, void* out, float* lse, void* stream,
+                        moda_impl impl) {
+    if (impl != MODA_IMPL_AUTO && impl != MODA_IMPL_SIMT && impl != MODA_IMPL_TC)
+        return MODA_ERR_INVALID_VALUE;
+    FwdArgs a;
+    moda_status st = fill_fwd(a, q, k, v, kd8, vd8, B, T, Hq, Hkv, d, Ld, dtype, scale, out, lse, false);
+    if (st != MODA_OK) return st;
+    if (Ld > 0) {
+        if (!kd_scale || !vd_scale) return MODA_ERR_INVALID_VALUE;
+        if ((reinterpret_cast<uintptr_t>(kd_scale) & 3u) || (reinterpret_cast<uintptr_t>(vd_scale) & 3u))
+            return MODA_ERR_MISALIGNED;
+        a.depth_q8 = 1;
+        a.kd_scale = kd_scale;
+        a.vd_scale = vd_scale;
+    }
+    return run_fwd(a, stream, impl);
+}
+
+namespace {
+moda_status check_q8_out(const int8_t* kd8, const int8_t* vd8, const float* ks, const float* vs) {
+    if (!kd8 || !vd8 || !ks || !vs) return MODA_ERR_INVALID_VALUE;
+    if ((reinterpret_cast<uintptr_t>(ks) & 3u) || (reinterpret_cast<uintptr_t>(vs) & 3u)) return MODA_ERR_MISALIGNED;
+    return MODA_OK;
+}
+}  // namespace
+
+moda_status moda_depth_quantize_q8(const void* kd, const void* vd, int B, int T, int Hkv, int d, int Ld,
+                                   moda_dtype dtype, int8_t* kd8, int8_t* vd8, float* kd_scale,
+                                   float* vd_scale, void* stream) {
+    if (B < 1 || T < 1 || Hkv < 1 || d < 1 || Ld < 0) return MODA_ERR_INVALID_VALUE;
+    if (dtype != MODA_BF16 && dtype != MODA_F32) return MODA_ERR_INVALID_VALUE;
+    if (d > 128) return MODA_ERR_UNSUPPORTED;
+    if (Ld == 0) return MODA_OK;
+    if (!kd || !vd) return MODA_ERR_INVALID_VALUE;
+    moda_status st = check_q8_out(kd8, vd8, kd_scale, vd_scale);
+    if (st != MODA_OK) return st;
+    const long long rows = (long long)B * T * Ld * Hkv;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_quantize_q8(kd, rows, d, dtype, 1, 1, 0, kd8, kd_scale, s);
+    if (e == cudaSuccess) e = launch_quantize_q8(vd, rows, d, dtype, 1, 1, 0, vd8, vd_scale, s);
+    return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
+}
+
+moda_status moda_depth_write_q8(const void* k, const void* v, int B, int T, int Hkv, int d, int Ld, int slot,
+                                moda_dtype dtype, int8_t* kd8, int8_t* vd8, float* kd_scale, float* vd_scale,
+                                void* stream) {
+    if (B < 1 || T < 1 || Hkv < 1 || d < 1 || Ld < 1) return MODA_ERR_INVALID_VALUE;
+    if (slot < 0 || slot >= Ld) return MODA_ERR_INVALID_VALUE;
+    if (dtype != MODA_BF16 && dtype != MODA_F32) return MODA_ERR_INVALID_VALUE;
+    if (d > 128) return MODA_ERR_UNSUPPORTED;
+    if (!k || !v) return MODA_ERR_INVALID_VALUE;
+    moda_status st = check_q8_out(kd8, vd8, kd_scale, vd_scale);
+    if (st != MODA_OK) return st;
+    // input row (b, t, h) -> depth row ((b*T + t)*Ld + slot)*Hkv + h
+    const long long rows = (long long)B * T * Hkv;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_quantize_q8(k, rows, d, dtype, Hkv, (long long)Ld * Hkv, (long long)slot * Hkv, kd8,
+                                       kd_scale, s);
+    if (e == cudaSuccess)
+        e = launch_quantize_q8(v, rows, d, dtype, Hkv, (long long)Ld * Hkv, (long long)slot * Hkv, vd8, vd_scale, s);
+    return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
+}
+
+moda_status moda_depth_slot_layout(int B, int T, int Hkv, int d, int Ld, int slot, long long* offset,
+                                   long long strides[4]) {
+    if (B < 1 || T < 1 || Hkv < 1 || d < 1 || Ld < 1 || slot < 0 || slot >= Ld) return MODA_ERR_INVALID_VALUE;
+    if (!offset || !strides) return MODA_ERR_INVALID_VALUE;
+    const Strides5 sd = strides_depth_native(T, Ld, Hkv, d);
+    *offset = (long long)slot * sd.si;
+    strides[0] = sd.sb;
+    strides[1] = sd.st;
+    strides[2] = sd.sh;
+    strides[3] = 1;
+    return MODA_OK;
+}
+
 moda_status moda_fwd_packed(const void* q, const void* k, const void* v, const void* packed_depth,
                             int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dtype,
                             float scale, void* out, float* lse, void* stream) {

@@ -85,6 +85,8 @@ struct TcFwdParams {
     float sl2;  // scale * log2(e)
     int depth_packed;
     const unsigned long long* depth_sel;  // [B,T] slot masks or null
+    const float* kd_scale;  // 8-bit depth: [B,T,Ld,Hkv] row scales (tm_kd / tm_vd map int8 codes)
+    const float* vd_scale;
     unsigned int* status;
     unsigned int wait_limit;
 };
@@ -93,6 +95,7 @@ struct __align__(8) Bars {
     uint64_t q_full;
     uint64_t full[kStages];
     uint64_t empty[kStages];
+    uint64_t raw_full[kStages];  // 8-bit depth tile landed (before dequantisation)
     uint64_t s_full[2];
     uint64_t p_full[2][4];  // [tile][P chunk]
     uint64_t o_final[2];
@@ -110,6 +113,63 @@ __device__ __forceinline__ void flag_timeout(TcFwdParams const& p, Bars* bars) {
     atomicOr(p.status, 1u);
 }
 
+// Ring use index of depth tile `seq` in stage `st`: how many earlier depth
+// tiles (sequence numbers >= first) used the same stage. Its parity is the
+// phase of raw_full[st] that marks this tile's arrival.
+__device__ __forceinline__ uint32_t depth_use(int seq, int first) {
+    const int st = seq % kStages;
+    const int f = first + ((st - first % kStages) + kStages) % kStages;
+    return (uint32_t)((seq - f) / kStages);
+}
+
+// 8-bit depth tiles: the producer's TMA puts a tile of 128 rows x 128 int8
+// codes as plain 128-byte lines into the second half of its ring slot; warps
+// 10 and 11 dequantise it in place into the bf16 128B-swizzled K-major layout
+// the MMA reads (row r: features 0-63 at r*128 of the first half, 64-127 at
+// r*128 of the second, 16-byte chunk j stored at chunk j ^ (r % 8)). A row's
+// second-half output overlaps only its own source line: each thread converts
+// its row in two passes, features 0-63 (written to the first half, which
+// holds no source) and then 64-127, whose source it reads before writing.
+// value = fp32(code * scale) rounded to bf16.
+__device__ __forceinline__ void dequant_row_q8(uint8_t* slot, int r, float sigma) {
+    const uint4* src = reinterpret_cast<const uint4*>(slot + kHalfBytes + r * 128);
+    const float2 bias = make_float2(-8388736.f, -8388736.f);  // 2^23 + 128
+    const float2 sg = make_float2(sigma, sigma);
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+    uint4 in[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) in[jj] = src[4 * pass + jj];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+        const int j = 4 * pass + jj;
+        const uint32_t w4[4] = {in[jj].x ^ 0x80808080u, in[jj].y ^ 0x80808080u, in[jj].z ^ 0x80808080u,
+                                in[jj].w ^ 0x80808080u};
+        uint32_t o[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            // code + 128 into the low byte of 2^23: the float 2^23 + code + 128
+            const float2 lo = make_float2(__uint_as_float(__byte_perm(w4[q], 0x4B000000u, 0x7540)),
+                                          __uint_as_float(__byte_perm(w4[q], 0x4B000000u, 0x7541)));
+            const float2 hi = make_float2(__uint_as_float(__byte_perm(w4[q], 0x4B000000u, 0x7542)),
+                                          __uint_as_float(__byte_perm(w4[q], 0x4B000000u, 0x7543)));
+            const float2 a = ptx::mul2(ptx::add2(lo, bias), sg);
+            const float2 b = ptx::mul2(ptx::add2(hi, bias), sg);
+            o[2 * q] = ptx::pack_bf16x2(a.x, a.y);
+            o[2 * q + 1] = ptx::pack_bf16x2(b.x, b.y);
+        }
+        // features 16j .. 16j+15 = output chunks 2j, 2j+1 (8 features each)
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int oc = 2 * j + u, h = oc >> 3, cj = oc & 7;
+            uint4* dst = reinterpret_cast<uint4*>(slot + h * kHalfBytes + r * 128 + ((cj ^ (r & 7)) << 4));
+            *dst = make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+        }
+    }
+    }
+}
+
+template <bool kQ8>
 __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_constant__ TcFwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -121,9 +181,12 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
     const uint32_t wait_limit = p.wait_limit;  // 0: time bound only
     volatile int* abort_flag = &bars->abort_flag;
 
-    // ---- work unit: heaviest (latest) token blocks first
-    const int bh = blockIdx.x % (p.B * p.Hkv);
-    const int tb = p.nblk - 1 - blockIdx.x / (p.B * p.Hkv);
+    // ---- work unit: (b, kv-head)-major, heaviest (latest) token blocks
+    // first within each. CTAs in flight then share one kv-head's K/V stream
+    // in L2 (at T = 64K one head's K + V is 32 MB; all four heads' streams
+    // together exceed the 126 MB L2), and the lightest blocks come last.
+    const int bh = blockIdx.x / p.nblk;
+    const int tb = p.nblk - 1 - blockIdx.x % p.nblk;
     const int b = bh / p.Hkv, kvh = bh % p.Hkv;
     const int n = p.n;
     const int t0 = tb * 2 * n;
@@ -155,6 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(&bars->full[s], 1);
             ptx::mbar_init(&bars->empty[s], 1);
+            ptx::mbar_init(&bars->raw_full[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&bars->s_full[i], 1);
@@ -207,8 +271,16 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                     ok = false;
                     break;
                 }
-                ptx::mbar_arrive_expect_tx_lead(&bars->full[st], kTileBytes, lead);
                 uint8_t* dst = sRing + st * kTileBytes;
+                if (kQ8 && x >= n_seq) {
+                    // int8 codes into the slot's second half; warps 10-11
+                    // dequantise them and complete full[st]
+                    ptx::mbar_arrive_expect_tx_lead(&bars->raw_full[st], kHalfBytes, lead);
+                    ptx::tma_load_4d_lead(dst + kHalfBytes, kv ? &p.tm_vd : &p.tm_kd, &bars->raw_full[st], 0, kvh,
+                                          t0 * p.Ld + (x - n_seq) * kBN, b, lead);
+                    continue;
+                }
+                ptx::mbar_arrive_expect_tx_lead(&bars->full[st], kTileBytes, lead);
                 for (int hf = 0; hf < 2; ++hf) {
                     if (x < n_seq) {
                         ptx::tma_load_4d_lead(dst + hf * kHalfBytes, kv ? &p.tm_v : &p.tm_k, &bars->full[st], hf * 64,
@@ -226,8 +298,12 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
         }
         // Drain: every load this CTA issued lands before the CTA can exit.
         ptx::mbar_wait(&bars->q_full, 0, kNoPollLimit, nullptr);
-        for (int s = (seq > kStages ? seq - kStages : 0); s < seq; ++s)
-            ptx::mbar_wait(&bars->full[s % kStages], (s / kStages) & 1, kNoPollLimit, nullptr);
+        for (int s = (seq > kStages ? seq - kStages : 0); s < seq; ++s) {
+            if (kQ8 && s >= 2 * n_seq)
+                ptx::mbar_wait(&bars->raw_full[s % kStages], depth_use(s, 2 * n_seq) & 1, kNoPollLimit, nullptr);
+            else
+                ptx::mbar_wait(&bars->full[s % kStages], (s / kStages) & 1, kNoPollLimit, nullptr);
+        }
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // One thread runs the MMA schedule: a tcgen05.mma issued by a single
@@ -335,6 +411,36 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
             ptx::mbar_wait(&bars->drain, 0, kNoPollLimit, nullptr);
         }
         __syncwarp();
+    } else if (kQ8 && warp >= 10) {
+        // ------------------------------------ 8-bit depth: dequantisation
+        const int ct = threadIdx.x - 10 * 32;  // 0..63: rows ct and ct + 64
+        const long long srow0 = (long long)b * p.T * p.Ld;
+        for (int x = n_seq; x < n_items; ++x) {
+            const int row0 = t0 * p.Ld + (x - n_seq) * kBN;  // first depth row of the tile
+            for (int kv = 0; kv < 2; ++kv) {
+                const int seq = 2 * x + kv, st = seq % kStages;
+                const float* scl = kv ? p.vd_scale : p.kd_scale;
+                float sg[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int row = row0 + ct + 64 * u;
+                    sg[u] = row < p.T * p.Ld ? __ldg(scl + (srow0 + row) * p.Hkv + kvh) : 0.f;
+                }
+                const bool got = ptx::mbar_wait(&bars->raw_full[st], depth_use(seq, 2 * n_seq) & 1, wait_limit,
+                                                abort_flag);
+                if (!ptx::bar_and(1, 64, got)) {
+                    if (ct == 0) flag_timeout(p, bars);
+                    x = n_items;
+                    break;
+                }
+                uint8_t* slot = sRing + st * kTileBytes;
+                dequant_row_q8(slot, ct, sg[0]);
+                dequant_row_q8(slot, ct + 64, sg[1]);
+                ptx::fence_proxy_async_smem();  // generic-proxy writes -> tensor core
+                ptx::bar_sync(1, 64);
+                if (ct == 0) ptx::mbar_arrive(&bars->full[st]);
+            }
+        }
     } else if (warp < 8) {
         // ------------------------------------------------ softmax warpgroups
         ptx::setmaxnreg_inc<kSoftmaxRegs>();
@@ -554,8 +660,16 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s) {
         if (!make_tmap_bf16_4d(&p.tm_k, a.k, dims, st, box)) return cudaErrorInvalidValue;
         if (!make_tmap_bf16_4d(&p.tm_v, a.v, dims, st, box)) return cudaErrorInvalidValue;
     }
-    const bool packed = a.Ld > 0 && a.sdep.si == kD;  // [B, Hkv, T*Ld, d]
-    if (a.Ld > 0) {
+    const bool packed = a.Ld > 0 && !a.depth_q8 && a.sdep.si == kD;  // [B, Hkv, T*Ld, d]
+    if (a.Ld > 0 && a.depth_q8) {
+        // int8 codes, [B, T*Ld, Hkv, 128] bytes
+        const cuuint64_t rows = (cuuint64_t)a.T * a.Ld;
+        const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)a.Hkv, rows, (cuuint64_t)a.B};
+        const cuuint64_t st[3] = {(cuuint64_t)kD, (cuuint64_t)a.Hkv * kD, rows * a.Hkv * kD};
+        const cuuint32_t box[4] = {(cuuint32_t)kD, 1, (cuuint32_t)kBN, 1};
+        if (!make_tmap_u8_4d(&p.tm_kd, a.kd, dims, st, box)) return cudaErrorInvalidValue;
+        if (!make_tmap_u8_4d(&p.tm_vd, a.vd, dims, st, box)) return cudaErrorInvalidValue;
+    } else if (a.Ld > 0) {
         const cuuint64_t rows = (cuuint64_t)a.T * a.Ld;
         if (packed) {
             const cuuint64_t dims[4] = {(cuuint64_t)kD, rows, (cuuint64_t)a.Hkv, (cuuint64_t)a.B};
@@ -581,13 +695,17 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s) {
     p.sl2 = a.scale * 1.4426950408889634f;
     p.depth_packed = packed ? 1 : 0;
     p.depth_sel = a.depth_sel;
+    p.kd_scale = a.kd_scale;
+    p.vd_scale = a.vd_scale;
     p.status = a.status;
     p.wait_limit = a.wait_limit;
-    cudaError_t err = cudaFuncSetAttribute(moda_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    const bool q8 = a.Ld > 0 && a.depth_q8;
+    auto kern = q8 ? moda_fwd_tc_kernel<true> : moda_fwd_tc_kernel<false>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
     const long long grid = (long long)p.nblk * a.B * a.Hkv;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
-    moda_fwd_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(p);
+    kern<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -34,6 +34,11 @@ struct FwdArgs {
     Strides5 sdep;    // kd and vd share strides
     moda_dtype dtype;
     const unsigned long long* depth_sel;  // [B,T] depth-slot bit masks, or null (all slots)
+    // 8-bit depth KV: kd / vd hold int8 codes [B,T,Ld,Hkv,d] and the depth
+    // values are scale * code with one fp32 scale per (b,t,i,kvh) row
+    int depth_q8;
+    const float* kd_scale;    // [B,T,Ld,Hkv]
+    const float* vd_scale;
     unsigned int* status;     // device status word
     unsigned int wait_limit;  // bounded-wait polls (0 = kernel default)
 };
@@ -76,6 +81,12 @@ cudaError_t launch_pack_depth(const void* kd, const void* vd, int B, int T, int 
                               int Ld, moda_dtype dt, void* packed, cudaStream_t s);
 cudaError_t launch_depth_write(const void* k, const void* v, int B, int T, int Hkv, int d, int Ld,
                                int slot, moda_dtype dt, void* kd, void* vd, cudaStream_t s);
+// Per-row int8 quantisation of `rows` rows of d values (input dtype dt):
+// input row r -> output row (r / inner) * out_tok_stride + out_off + r % inner
+// of codes [*, d] and scales [*].
+cudaError_t launch_quantize_q8(const void* x, long long rows, int d, moda_dtype dt, int inner,
+                               long long out_tok_stride, long long out_off, int8_t* codes,
+                               float* scales, cudaStream_t s);
 
 // Tensor-core kernels for sm_100a (moda_fwd_sm100.cu, moda_bwd_sm100.cu).
 bool fwd_tc_supported(const FwdArgs& a);

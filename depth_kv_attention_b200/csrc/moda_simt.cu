@@ -32,6 +32,9 @@ __device__ __forceinline__ float to_f<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
 
+template <>
+__device__ __forceinline__ float to_f<int8_t>(int8_t x) { return (float)x; }
+
 template <typename T>
 __device__ __forceinline__ T from_f(float x);
 template <>
@@ -62,6 +65,19 @@ __device__ __forceinline__ void load_row(const T* row, int d, int u, float2 (&r)
         const int c = Split<TPR>::feat(i, u);
         r[i].x = (c < d) ? to_f(row[c]) * mul : 0.f;
         r[i].y = (c + 1 < d) ? to_f(row[c + 1]) * mul : 0.f;
+    }
+}
+
+// 8-bit depth row: fl32(scale * code), then rounded to the input dtype T
+// (the type the unquantised depth cache would hold).
+template <int TPR, typename T>
+__device__ __forceinline__ void load_row_q8(const int8_t* row, int d, int u, float2 (&r)[Split<TPR>::NP],
+                                            float sigma) {
+    load_row<TPR>(row, d, u, r, sigma);
+#pragma unroll
+    for (int i = 0; i < Split<TPR>::NP; ++i) {
+        r[i].x = to_f(from_f<T>(r[i].x));
+        r[i].y = to_f(from_f<T>(r[i].y));
     }
 }
 
@@ -169,11 +185,18 @@ __global__ void __launch_bounds__(128) fwd_simt_kernel(FwdArgs a, int n_tok, int
     for (int i = 0; i < a.Ld; ++i) {
         const long long off = b * a.sdep.sb + tc * a.sdep.st + (long long)i * a.sdep.si + kvh * a.sdep.sh;
         float2 kr[S::NP];
-        load_row<TPR>(KD + off, a.d, u, kr);
+        const long long srow = off / a.d;  // (b, t, i, kvh) row of the 8-bit scales
+        if (a.depth_q8)
+            load_row_q8<TPR, T>(static_cast<const int8_t*>(a.kd) + off, a.d, u, kr, a.kd_scale[srow]);
+        else
+            load_row<TPR>(KD + off, a.d, u, kr);
         const float s = group_sum<TPR>(dot_regs<TPR>(q, kr));
         if (a.depth_sel && !((sel >> i) & 1ull)) continue;
         float2 vr[S::NP];
-        load_row<TPR>(VD + off, a.d, u, vr);
+        if (a.depth_q8)
+            load_row_q8<TPR, T>(static_cast<const int8_t*>(a.vd) + off, a.d, u, vr, a.vd_scale[srow]);
+        else
+            load_row<TPR>(VD + off, a.d, u, vr);
         if (s > m) {
             const float corr = exp2f(m - s);
             l *= corr;
@@ -559,6 +582,60 @@ cudaError_t launch_depth_write(const void* k, const void* v, int B, int T, int H
     depth_write_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v),
                                                         static_cast<uint4*>(kd), static_cast<uint4*>(vd), rows,
                                                         row_vec, Ld, slot);
+    return cudaGetLastError();
+}
+
+namespace {
+// 8-bit depth KV: one warp per row of d <= 128 values. amax over the row,
+// scale = amax / 127 and code = round-half-even(x / scale) clamped to
+// [-127, 127], each a single IEEE fp32 operation (__fdiv_rn, __float2int_rn)
+// so the codes are exactly those of the float32 definition; an all-zero row
+// gets scale 0 and codes 0.
+template <typename T>
+__global__ void quantize_q8_kernel(const T* x, long long rows, int d, int inner, long long out_tok_stride,
+                                   long long out_off, int8_t* codes, float* scales) {
+    const long long r = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    if (r >= rows) return;
+    const int lane = threadIdx.x % 32;
+    const T* row = x + r * d;
+    float v[4];
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int c = lane + 32 * e;
+        v[e] = c < d ? to_f(row[c]) : 0.f;
+        amax = fmaxf(amax, fabsf(v[e]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float sigma = __fdiv_rn(amax, 127.f);
+    const long long orow = (r / inner) * out_tok_stride + out_off + r % inner;
+    int8_t* crow = codes + orow * d;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int c = lane + 32 * e;
+        if (c < d) {
+            int q = 0;
+            if (sigma > 0.f) q = min(127, max(-127, __float2int_rn(__fdiv_rn(v[e], sigma))));
+            crow[c] = (int8_t)q;
+        }
+    }
+    if (lane == 0) scales[orow] = sigma;
+}
+}  // namespace
+
+cudaError_t launch_quantize_q8(const void* x, long long rows, int d, moda_dtype dt, int inner,
+                               long long out_tok_stride, long long out_off, int8_t* codes,
+                               float* scales, cudaStream_t s) {
+    if (rows <= 0) return cudaSuccess;
+    const long long blocks = (rows + 7) / 8;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+    if (dt == MODA_F32)
+        quantize_q8_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const float*>(x), rows, d, inner,
+                                                                    out_tok_stride, out_off, codes, scales);
+    else
+        quantize_q8_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(x), rows, d, inner, out_tok_stride, out_off, codes, scales);
     return cudaGetLastError();
 }
 

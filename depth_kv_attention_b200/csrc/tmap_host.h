@@ -36,4 +36,17 @@ inline bool make_tmap_bf16_4d(CUtensorMap* m, const void* base, const cuuint64_t
     return r == CUDA_SUCCESS;
 }
 
+// 4-D map of bytes (8-bit depth codes) without swizzle: rows land in shared
+// memory as plain 128-byte lines for the in-place dequantisation.
+inline bool make_tmap_u8_4d(CUtensorMap* m, const void* base, const cuuint64_t dims[4],
+                            const cuuint64_t strides_b[3], const cuuint32_t box[4]) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides_b, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace moda

@@ -270,6 +270,66 @@ moda_status moda_depth_write(const void* k, const void* v,
                              int B, int T, int Hkv, int d, int Ld, int slot,
                              moda_dtype dtype, void* kd, void* vd, void* stream);
 
+/*
+ * 8-bit depth KV. "动态混合深度注意力机制MoDA技术解析" (mhpn.cn) §4.2 suggests
+ * storing the depth KV of deep models (beyond 32 layers) with 8-bit
+ * quantisation where device memory is short; the page names no format. This
+ * library's format: int8 codes in the native depth layout [B,T,Ld,Hkv,d] and
+ * one fp32 scale per (b, t, slot, kv-head) row of d values [B,T,Ld,Hkv]:
+ *     scale = amax / 127 (amax = max |x| over the row; 0 for a zero row),
+ *     code  = round-half-even(x / scale) clamped to [-127, 127]  (0 if scale 0),
+ * each step one IEEE fp32 operation. The depth value the forward attends to
+ * is fp32(scale * code) rounded to the input dtype (round to nearest even
+ * for bf16): the 8-bit cache decompresses into the type an unquantised depth
+ * cache would hold. About half the bytes of the bf16 depth stream (d + 4
+ * bytes per row instead of 2d).
+ *
+ * moda_depth_quantize_q8 — quantise a whole bf16 / fp32 depth cache.
+ *   kd, vd [B,T,Ld,Hkv,d]             in   (input dtype)
+ *   kd8, vd8 [B,T,Ld,Hkv,d] int8      out  16-byte aligned
+ *   kd_scale, vd_scale [B,T,Ld,Hkv]   out  fp32, 4-byte aligned
+ * moda_depth_write_q8 — the write step into an 8-bit cache: k, v [B,T,Hkv,d]
+ *   quantised into slot `slot` (0 <= slot < Ld) of kd8 / vd8 and its scales;
+ *   other slots untouched.
+ * moda_fwd_q8 — moda_fwd_ex reading the 8-bit depth cache (codes and
+ *   scales as above; all four may be NULL iff Ld == 0). The tensor-core path
+ *   dequantises each depth tile in shared memory, the SIMT path per row in
+ *   registers, to the same values. Forward only: there is no 8-bit backward.
+ * Errors as moda_fwd_ex / moda_depth_write; MODA_ERR_MISALIGNED for a scale
+ * pointer that is not 4-byte aligned.
+ */
+moda_status moda_depth_quantize_q8(const void* kd, const void* vd,
+                                   int B, int T, int Hkv, int d, int Ld, moda_dtype dtype,
+                                   int8_t* kd8, int8_t* vd8, float* kd_scale, float* vd_scale,
+                                   void* stream);
+moda_status moda_depth_write_q8(const void* k, const void* v,
+                                int B, int T, int Hkv, int d, int Ld, int slot, moda_dtype dtype,
+                                int8_t* kd8, int8_t* vd8, float* kd_scale, float* vd_scale,
+                                void* stream);
+moda_status moda_fwd_q8(const void* q, const void* k, const void* v,
+                        const int8_t* kd8, const int8_t* vd8,
+                        const float* kd_scale, const float* vd_scale,
+                        int B, int T, int Hq, int Hkv, int d, int Ld,
+                        moda_dtype dtype, float scale,
+                        void* out, float* lse, void* stream, moda_impl impl);
+
+/*
+ * moda_depth_slot_layout — where a producer writes a layer's K / V so that
+ * they land directly in slot `slot` of the native depth cache, with no copy
+ * pass: the write step of "Mixture-of-Depths Attention" (gist.science German
+ * summary §2, Write-Step) fused into whatever kernel produces the pair (the
+ * layer's key / value projection, or an FFN layer's light projection).
+ * Slot `slot` of kd [B,T,Ld,Hkv,d] is the strided tensor [B, T, Hkv, d] that
+ * starts `*offset` elements after kd and has element strides
+ *     strides[0..3] = {T*Ld*Hkv*d, Ld*Hkv*d, d, 1}     (b, t, h, feature)
+ * so a GEMM producing the [B*T, Hkv*d] row block writes it with leading
+ * dimension Ld*Hkv*d (vd likewise). moda_depth_write is the copy pass this
+ * replaces. Returns MODA_ERR_INVALID_VALUE for a bad shape, slot or NULL
+ * output pointer; touches no device.
+ */
+moda_status moda_depth_slot_layout(int B, int T, int Hkv, int d, int Ld, int slot,
+                                   long long* offset, long long strides[4]);
+
 /* moda_fwd reading depth keys/values from moda_pack_depth's layout. */
 moda_status moda_fwd_packed(const void* q, const void* k, const void* v,
                             const void* packed_depth,

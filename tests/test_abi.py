@@ -145,3 +145,35 @@ def test_fwd_host_staging_size_and_validation():
     assert fwd_host(q=None) == 1
     assert fwd_host(Hq=3) == 1
     assert fwd_host(d=256) == 2
+
+
+def test_q8_validation():
+    """8-bit depth entry points: NULL / misaligned scales and codes, slots
+    outside [0, Ld), unsupported d."""
+    fq = lambda ks=P, kd8=P, Ld=2: moda._c_fwd_q8(P, P, P, kd8, P, ks, P, 1, 8, 4, 2, 64, Ld, 0, 0.125,  # noqa: E731
+                                                   P, P, None, 0)
+    assert fq(ks=None) == 1
+    assert fq(ks=P + 2) == 3
+    assert fq(kd8=P + 8) == 3
+    assert fq(kd8=None) == 1
+    qz = lambda kd8=P, ks=P, d=64: moda._c_quant_q8(P, P, 1, 4, 2, d, 2, 0, kd8, P, ks, P, None)  # noqa: E731
+    assert qz(kd8=None) == 1
+    assert qz(ks=P + 1) == 3
+    assert qz(d=256) == 2
+    wq = lambda slot=0, Ld=2: moda._c_write_q8(P, P, 1, 4, 2, 64, Ld, slot, 0, P, P, P, P, None)  # noqa: E731
+    assert wq(slot=2) == 1
+    assert wq(slot=-1) == 1
+    assert wq(Ld=0) == 1
+
+
+def test_slot_layout_is_the_native_slot():
+    import torch
+    """moda_depth_slot_layout's offset and strides address exactly
+    kd[:, :, slot] of the native cache (CPU: a view on a host tensor)."""
+    kd = torch.arange(2 * 5 * 3 * 2 * 4).reshape(2, 5, 3, 2, 4)
+    for slot in range(3):
+        assert torch.equal(moda.depth_slot_view(kd, slot), kd[:, :, slot])
+    assert moda.moda_depth_slot_layout(2, 5, 2, 4, 3, 1) == (8, (120, 24, 4, 1))
+    with pytest.raises(moda.ModaError):
+        moda.moda_depth_slot_layout(2, 5, 2, 4, 3, 3)
+

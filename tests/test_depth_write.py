@@ -61,3 +61,46 @@ def test_depth_written_layer_by_layer_then_forward():
     ro, rl = oracle.forward(x["q"], x["k"], x["v"], sk, sv, w.scale)
     compare("write-then-read out", f64(out), ro, "bf16")
     compare("write-then-read lse", f64(lse), rl, "bf16", what="lse")
+
+
+def test_producer_writes_straight_into_depth_slots():
+    """The write step fused with its producer: each earlier layer's key and
+    value projections (GEMMs x_l @ W) write their [B*T, Hkv*d] output directly
+    into slot l of the native depth cache through the slot view (leading
+    dimension Ld*Hkv*d). No copy or elementwise kernel runs while the cache is
+    filled, the slots hold the projections, and the forward over the cache
+    matches the oracle."""
+    B, T, Hq, Hkv, d, Ld, Dm = 2, 300, 16, 2, 128, 3, 256
+    g = torch.Generator("cpu")
+    g.manual_seed(23)
+    dt = torch.bfloat16
+    xs = [torch.randn(B * T, Dm, generator=g).to(dt).cuda() for _ in range(Ld)]
+    wk = [(torch.randn(Dm, Hkv * d, generator=g) / 16).to(dt).cuda() for _ in range(Ld)]
+    wv = [(torch.randn(Dm, Hkv * d, generator=g) / 16).to(dt).cuda() for _ in range(Ld)]
+    q = torch.randn(B, T, Hq, d, generator=g).to(dt).cuda()
+    k = torch.randn(B, T, Hkv, d, generator=g).to(dt).cuda()
+    v = torch.randn(B, T, Hkv, d, generator=g).to(dt).cuda()
+    kd = torch.zeros(B, T, Ld, Hkv, d, dtype=dt, device="cuda")
+    vd = torch.zeros_like(kd)
+    torch.cuda.synchronize()
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        for layer in range(Ld):
+            for cache, w in ((kd, wk[layer]), (vd, wv[layer])):
+                view = moda.depth_slot_view(cache, layer).view(B * T, Hkv * d)  # stride (Ld*Hkv*d, 1)
+                torch.mm(xs[layer], w, out=view)
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events() if e.device_type.name == "CUDA"]
+    assert names, "no kernel recorded"
+    bad = [n for n in names if any(s in n.lower() for s in ("copy", "elementwise", "memcpy", "fill"))]
+    assert not bad, bad
+    for layer in range(Ld):
+        want_k = (xs[layer] @ wk[layer]).view(B, T, Hkv, d)
+        want_v = (xs[layer] @ wv[layer]).view(B, T, Hkv, d)
+        torch.testing.assert_close(kd[:, :, layer], want_k, rtol=1e-2, atol=1e-2)
+        torch.testing.assert_close(vd[:, :, layer], want_v, rtol=1e-2, atol=1e-2)
+    out, lse = moda.moda_fwd(q, k, v, kd, vd)
+    torch.cuda.synchronize()
+    ro, rl = oracle.forward(q.cpu(), k.cpu(), v.cpu(), kd.cpu(), vd.cpu(), 1.0 / d ** 0.5)
+    compare("strided-producer cache out", f64(out), ro, "bf16")
+    compare("strided-producer cache lse", f64(lse), rl, "bf16", what="lse")
