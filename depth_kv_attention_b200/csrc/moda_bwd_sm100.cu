@@ -9,17 +9,17 @@
 //   dkd_i = scale sum_h dS'_i q,  dvd_i = sum_h P'_i dout   (same token)
 //
 // Launch sequence (one stream):
-//   1. D~ = rowsum(dout * out), an estimate of D from the stored output (SIMT)
-//   2. dq: query-major tensor-core kernel over the causal key tiles and the
-//      query tile's own depth chunks. It sees all keys of its rows, so it
-//      also forms the exact D = D~ + sum_j P_j (dP_j - D~) and corrects dq
-//      for D - D~; dq accumulates in TMEM and is written once, in bf16
-//   3. dk, dv: KV-major tensor-core kernel (reads the exact D); partial sums
+//   1. dq: query-major tensor-core kernel over the causal key tiles and the
+//      query tile's own depth chunks. It forms the estimate D~ = <dout, out>
+//      from the stored output, sees all keys of its rows, and so also forms
+//      the exact D = D~ + sum_j P_j (dP_j - D~) and corrects dq for D - D~;
+//      dq accumulates in TMEM and is written once, in bf16
+//   2. dk, dv: KV-major tensor-core kernel (reads the exact D); partial sums
 //      of a key tile over a chunk of query tiles go to fp32 accumulators
 //      with vector reductions
-//   4. dkd, dvd: the same kernel with 128-row depth chunks as the key tiles
+//   3. dkd, dvd: the same kernel with 128-row depth chunks as the key tiles
 //      and a same-token mask (each depth row owned by one CTA, bf16 stores)
-//   5. dk, dv = bf16(accumulators)
+//   4. dk, dv = bf16(accumulators)
 // Splitting dq from dk/dv recomputes S and dP once more but removes the
 // per-pair fp32 dq reductions, which for wide GQA (G = 32, 4 tokens per
 // 128-row tile) would move gigabytes through L2.
@@ -105,7 +105,7 @@ struct __align__(8) Bars {
     uint64_t kv_full;            // dk/dv kernel: K, V tile | dq kernel: Q, dO tile
     uint64_t full[4];            // ring slots
     uint64_t empty[4];
-    uint64_t s_full, dp_full, p_full, p_full2, fin, drain;
+    uint64_t s_full, dp_full, p_full, p_full2, fin, drain, dp_read;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -130,6 +130,7 @@ __device__ __forceinline__ void init_bars(Bars* bars, int stages, int p_count) {
     ptx::mbar_init(&bars->p_full2, p_count);
     ptx::mbar_init(&bars->fin, 1);
     ptx::mbar_init(&bars->drain, 1);
+    ptx::mbar_init(&bars->dp_read, 8);
     bars->abort_flag = 0;
     ptx::fence_barrier_init();
     ptx::fence_proxy_async_smem();
@@ -505,8 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
 struct DqParams {
     CUtensorMap tm_q, tm_do, tm_k, tm_v, tm_kd, tm_vd;
     const float* lse;
-    float* rowD;  // in: D~ = <dout, out> per row; out: D = sum_j P_j dP_j
+    float* rowD;  // out: D = sum_j P_j dP_j per row, for the dK/dV kernels
     void* dq;     // [B,T,Hq,d] bf16
+    const void* dout;  // [B,T,Hq,d] bf16 \ for D~ = <dout, out>, formed
+    const void* out;   // [B,T,Hq,d] bf16 / at the start
     const unsigned long long* depth_sel;  // [B,T] slot masks or null
     int B, T, Hq, Hkv, G, n, Ld, nqt;
     float sl2, scale;
@@ -526,8 +529,8 @@ static_assert(kDqSmem <= 232448, "shared memory per CTA");
 // output the forward stored is rounded to bf16 (and was formed from bf16 P),
 // and wide depth keys amplify that rounding through dq = scale sum dS k by
 // |kd|. This kernel sees every key of its rows, so it computes D itself:
-// with the estimate D~ = <dout, out> (the first kernel of the backward) it
-// forms dS~ = P (dP - D~) in fp32 and accumulates, per row,
+// with the estimate D~ = <dout, out> (formed from the stored output at the
+// start) it forms dS~ = P (dP - D~) in fp32 and accumulates, per row,
 //   delta = sum_j dS~_j   (= D - D~, since sum_j P_j = 1),
 //   dQ~  += dS~ K          (bf16 dS~: the near-cancellation dP - D~ is fp32)
 //   Bq   += P K            (the attention-weighted mean key)
@@ -544,15 +547,21 @@ static_assert(kDqSmem <= 232448, "shared memory per CTA");
 // R[x % 2] and dP(x) in R[(x + 1) % 2]. The compute warps write P(x) and
 // dS~(x) in bf16 over S(x) (each column half: dS~ at its columns 0-31, P at
 // 32-63; for a depth item the lo term of dS~ over the half's dP columns
-// 0-31, already read); once they publish them the MMA warp issues, in this
-// order (tcgen05.mma operations of one CTA execute in issue order):
-//   S(x+1) = Q K(x+1)^T   into R[(x+1) % 2] (dP(x) there has been read)
-//   dQ~   += dS~(x) K(x)  A = dS~(x) from R[x % 2]
-//   Bq    += P(x) K(x)    A = P(x) from R[x % 2]
+// 0-31, already read). The MMA warp issues, in this order (tcgen05.mma
+// operations of one CTA execute in issue order):
+//   S(x+1) = Q K(x+1)^T   into R[(x+1) % 2], as soon as the compute warps
+//                         have loaded dP(x) from there (dp_read, before they
+//                         form dS~(x))
+//   dQ~   += dS~(x) K(x)  A = dS~(x) from R[x % 2]  \ once dS~(x) and P(x)
+//   Bq    += P(x) K(x)    A = P(x) from R[x % 2]    / are written (p_full)
 //   dP(x+1) = dO V(x+1)^T into R[x % 2], after both have read it
-// so the compute warps exponentiate S(x+1) while these run, then form
-// dS~(x+1). A depth item issues dQ~ += lo(x) K(x) (A from R[(x+1) % 2]) after
-// dQ~ and Bq, and S(x+1) only after that.
+// so S(x+1) runs while the compute warps form dS~(x), and the compute warps
+// exponentiate S(x+1) while dQ~, Bq and dP(x+1) run. A depth item issues
+// dQ~ += lo(x) K(x) (A from R[(x+1) % 2]) after dQ~ and Bq, and S(x+1) only
+// after that.
+// Measured against two other arrangements on the wide-GQA workload (8192
+// tokens, G = 32): S(x+1) only after dS~(x) (1.23 ms) and P / dS~ in shared
+// memory with SS MMAs and dO in TMEM (1.42 ms) against 1.21 ms for this one.
 __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_constant__ DqParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -670,17 +679,32 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
             };
             if (ok) ok = issue_s(0) && issue_dp(0);
             for (int x = 0; x < n_items && ok; ++x) {
-                // dS(x) is in R[x % 2]; the compute warps have read dP(x) from
-                // R[(x + 1) % 2], which S(x + 1) may now overwrite.
-                if (!wait_one(&bars->p_full, x & 1)) {
+                // the compute warps have read dP(x) from R[(x + 1) % 2], which
+                // S(x + 1) may now overwrite (depth items: after the lo MMA)
+                if (!wait_one(&bars->dp_read, x & 1)) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
+                if (x >= n_kv) {
+                    if (!wait_one(&bars->p_full, x & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                }
                 const bool depth_item = x >= n_kv;
                 if (!depth_item && x + 1 < n_items && !issue_s(x + 1)) {
                     ok = false;
                     break;
+                }
+                if (!depth_item) {
+                    // wait p_full only now: S(x+1) went out once dP(x) was read
+                    if (!wait_one(&bars->p_full, x & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
                 }
                 const int sk = 2 * x;
                 const uint64_t km = mndesc(aRing + (sk % kDqStages) * kTile);
@@ -727,11 +751,33 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
         const int tt = r / p.G;          // token within the tile
         const int t = t0 + tt, h = kvh * p.G + r % p.G;
         const bool row_ok = t < p.T;
-        float lse2 = INFINITY, Drow = 0.f;
-        if (row_ok) {
-            const long long ix = ((long long)b * p.Hq + h) * p.T + t;
-            lse2 = p.lse[ix] * kLog2e;
-            Drow = p.rowD[ix];
+        float lse2 = INFINITY;
+        if (row_ok) lse2 = p.lse[((long long)b * p.Hq + h) * p.T + t] * kLog2e;
+        // D~ = <dout, out> of the row from the stored output: each column half
+        // sums its 64 features, and the halves add through shared memory
+        // (sDelta is written again only after the item loop, which no thread
+        // finishes before every thread has passed this point: each item
+        // needs the arrivals of all 256 compute threads)
+        float Drow;
+        {
+            const long long roff = (((long long)b * p.T + (row_ok ? t : 0)) * p.Hq + h) * kD + 64 * hs;
+            const uint4* du = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dout) + roff);
+            const uint4* ou = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.out) + roff);
+            float part = 0.f;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const uint4 u = row_ok ? du[v] : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 o = row_ok ? ou[v] : make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t uw[4] = {u.x, u.y, u.z, u.w}, ow[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    part = fmaf(__uint_as_float(uw[q] << 16), __uint_as_float(ow[q] << 16), part);
+                    part = fmaf(__uint_as_float(uw[q] & 0xffff0000u), __uint_as_float(ow[q] & 0xffff0000u), part);
+                }
+            }
+            sDelta[hs * 128 + r] = part;
+            asm volatile("bar.sync 1, %0;" ::"n"(kComputeThreads) : "memory");
+            Drow = sDelta[r] + sDelta[128 + r];
         }
         const float sl2 = p.sl2;
         const bool has_sel = p.depth_sel != nullptr;
@@ -785,11 +831,17 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
             }
             ptx::tc_fence_after();
             const bool depth_item = x >= n_kv;
+            uint32_t drr[64];
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+                ptx::tmem_ld32(rP + 64 * hs + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&drr[32 * c]));
+            ptx::tmem_wait_ld();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&bars->dp_read);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                uint32_t dr[32];
-                ptx::tmem_ld32(rP + 64 * hs + 32 * c, dr);
-                ptx::tmem_wait_ld();
+                const uint32_t* dr = drr + 32 * c;
                 uint32_t dd[16], dl[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -890,8 +942,7 @@ bool bwd_tc_supported(const BwdArgs& a) {
 
 cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s) {
     const FwdArgs& f = a.f;
-    cudaError_t e = launch_bwd_rowdot(a, s);
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
     const int G = f.G, n = 128 / G;
     int gshift = 0;
     while ((1 << gshift) < G) ++gshift;
@@ -928,7 +979,7 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s) {
     DqParams pq;
     memset(&pq, 0, sizeof(pq));
     pq.tm_q = tm_q; pq.tm_do = tm_do; pq.tm_k = tm_k; pq.tm_v = tm_v; pq.tm_kd = tm_kd; pq.tm_vd = tm_vd;
-    pq.lse = f.lse; pq.rowD = a.rowD; pq.dq = a.dq;
+    pq.lse = f.lse; pq.rowD = a.rowD; pq.dq = a.dq; pq.dout = a.dout; pq.out = f.out;
     pq.B = f.B; pq.T = f.T; pq.Hq = f.Hq; pq.Hkv = f.Hkv; pq.G = G; pq.n = n; pq.Ld = f.Ld;
     pq.nqt = (f.T + n - 1) / n;
     pq.depth_sel = f.depth_sel;

@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&bars->s_full[i], 1);
-            for (int c = 0; c < kPChunks; ++c) ptx::mbar_init(&bars->p_full[i][c], 128);
+            for (int c = 0; c < kPChunks; ++c) ptx::mbar_init(&bars->p_full[i][c], 4);  // one per warp
             ptx::mbar_init(&bars->o_final[i], 1);
         }
         ptx::mbar_init(&bars->drain, 1);
@@ -562,7 +562,10 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                     ptx::tmem_st16(tS + ch * kPairs + q * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[q * 16]));
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(&bars->p_full[i][ch]);
+                // one arrival per warp: 128 per-thread arrivals on one
+                // barrier word serialise on the tile's critical chain
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&bars->p_full[i][ch]);
             }
             {
                 const float2 a01 = ptx::add2(acc[0], acc[1]), a23 = ptx::add2(acc[2], acc[3]);

@@ -73,10 +73,6 @@ inline Strides5 strides_depth_packed(int T, int Ld, int Hkv, int d) {
 // SIMT kernels (moda_simt.cu). Any d <= 128, any G, fp32 or bf16.
 cudaError_t launch_fwd_simt(const FwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t s);
-// Pieces of the SIMT backward that the tensor-core backward reuses:
-// D = rowsum(dout * out) into a.rowD, and dkd / dvd.
-cudaError_t launch_bwd_rowdot(const BwdArgs& a, cudaStream_t s);
-cudaError_t launch_bwd_depth_dkv(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_pack_depth(const void* kd, const void* vd, int B, int T, int Hkv, int d,
                               int Ld, moda_dtype dt, void* packed, cudaStream_t s);
 cudaError_t launch_depth_write(const void* k, const void* v, int B, int T, int Hkv, int d, int Ld,

@@ -531,24 +531,6 @@ cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_rowdot(const BwdArgs& a, cudaStream_t s) {
-    const long long rows = (long long)a.f.B * a.f.T * a.f.Hq;
-    dim3 grid((unsigned)((rows + 7) / 8));
-    if (a.f.dtype == MODA_F32) bwd_rowdot_kernel<float><<<grid, 256, 0, s>>>(a);
-    else bwd_rowdot_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_bwd_depth_dkv(const BwdArgs& a, cudaStream_t s) {
-    const FwdArgs& f = a.f;
-    if (f.Ld == 0) return cudaSuccess;
-    const long long items = (long long)f.B * f.T * f.Ld * f.Hkv;
-    dim3 grid((unsigned)((items + 63) / 64));
-    if (f.dtype == MODA_F32) bwd_depth_simt_kernel<float><<<grid, 256, 0, s>>>(a);
-    else bwd_depth_simt_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
-    return cudaGetLastError();
-}
-
 // The write step: k / v [B,T,Hkv,d] into slot `slot` of kd / vd
 // [B,T,Ld,Hkv,d], 16-byte vectors. One (b, t) row of k is Hkv*vec vectors
 // and lands contiguously at kd[b, t, slot], so both sides stay coalesced.
