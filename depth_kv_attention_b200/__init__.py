@@ -35,7 +35,7 @@ lib = ctypes.CDLL(LIB_PATH)
 
 MODA_OK = 0
 _DTYPE = {torch.bfloat16: 0, torch.float32: 1}
-_IMPL = {"auto": 0, "simt": 1, "tc": 2}
+_IMPL = {"auto": 0, "simt": 1, "tc": 2, "tc2": 3}
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 
 

@@ -84,10 +84,12 @@ moda_status run_fwd(FwdArgs& a, void* stream, moda_impl impl) {
     cudaError_t e = status_ptr(&a.status, &a.wait_limit);
     if (e != cudaSuccess) return MODA_ERR_CUDA;
     const bool tc_ok = fwd_tc_supported(a);
-    if (impl == MODA_IMPL_TC && !tc_ok) return MODA_ERR_UNSUPPORTED;
-    const bool use_tc = impl == MODA_IMPL_TC || (impl == MODA_IMPL_AUTO && tc_ok);
+    if ((impl == MODA_IMPL_TC || impl == MODA_IMPL_TC2) && !tc_ok) return MODA_ERR_UNSUPPORTED;
+    if (impl == MODA_IMPL_TC2 && !fwd_pair_supported(a)) return MODA_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    e = use_tc ? launch_fwd_tc(a, s) : launch_fwd_simt(a, s);
+    if (impl == MODA_IMPL_SIMT || (impl == MODA_IMPL_AUTO && !tc_ok)) e = launch_fwd_simt(a, s);
+    else if (impl == MODA_IMPL_TC2) e = launch_fwd_pair(a, s);
+    else e = launch_fwd_tc(a, s);
     return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
 }
 
@@ -144,7 +146,7 @@ moda_status moda_fwd_sel(const void* q, const void* k, const void* v, const void
                          const void* vd, const uint64_t* depth_sel, int B, int T, int Hq, int Hkv,
                          int d, int Ld, moda_dtype dtype, float scale, void* out, float* lse,
                          void* stream, moda_impl impl) {
-    if (impl != MODA_IMPL_AUTO && impl != MODA_IMPL_SIMT && impl != MODA_IMPL_TC)
+    if (impl != MODA_IMPL_AUTO && impl != MODA_IMPL_SIMT && impl != MODA_IMPL_TC && impl != MODA_IMPL_TC2)
         return MODA_ERR_INVALID_VALUE;
     FwdArgs a;
     moda_status st = fill_fwd(a, q, k, v, kd, vd, B, T, Hq, Hkv, d, Ld, dtype, scale, out, lse, false);
@@ -182,7 +184,7 @@ moda_status moda_bwd_sel(const void* q, const void* k, const void* v, const void
                          int Ld, moda_dtype dtype, float scale, void* dq, void* dk, void* dv,
                          void* dkd, void* dvd, void* workspace, size_t workspace_bytes,
                          void* stream, moda_impl impl) {
-    if (impl != MODA_IMPL_AUTO && impl != MODA_IMPL_SIMT && impl != MODA_IMPL_TC)
+    if (impl != MODA_IMPL_AUTO && impl != MODA_IMPL_SIMT && impl != MODA_IMPL_TC && impl != MODA_IMPL_TC2)
         return MODA_ERR_INVALID_VALUE;
     BwdArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -209,8 +211,8 @@ moda_status moda_bwd_sel(const void* q, const void* k, const void* v, const void
     cudaError_t e = status_ptr(&a.f.status, &a.f.wait_limit);
     if (e != cudaSuccess) return MODA_ERR_CUDA;
     const bool tc_ok = bwd_tc_supported(a);
-    if (impl == MODA_IMPL_TC && !tc_ok) return MODA_ERR_UNSUPPORTED;
-    const bool use_tc = impl == MODA_IMPL_TC || (impl == MODA_IMPL_AUTO && tc_ok);
+    if ((impl == MODA_IMPL_TC || impl == MODA_IMPL_TC2) && !tc_ok) return MODA_ERR_UNSUPPORTED;
+    const bool use_tc = impl == MODA_IMPL_TC || impl == MODA_IMPL_TC2 || (impl == MODA_IMPL_AUTO && tc_ok);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     e = use_tc ? launch_bwd_tc(a, s) : launch_bwd_simt(a, s);
     return e == cudaSuccess ? MODA_OK : MODA_ERR_LAUNCH;
@@ -275,7 +277,7 @@ moda_status moda_fwd_q8(const void* q, const void* k, const void* v, const int8_
                         const float* kd_scale, const float* vd_scale, int B, int T, int Hq, int Hkv, int d,
                         int Ld, moda_dtype dtype, float scale, void* out, float* lse, void* stream,
                         moda_impl impl) {
-    if (impl != MODA_IMPL_AUTO && impl != MODA_IMPL_SIMT && impl != MODA_IMPL_TC)
+    if (impl != MODA_IMPL_AUTO && impl != MODA_IMPL_SIMT && impl != MODA_IMPL_TC && impl != MODA_IMPL_TC2)
         return MODA_ERR_INVALID_VALUE;
     FwdArgs a;
     moda_status st = fill_fwd(a, q, k, v, kd8, vd8, B, T, Hq, Hkv, d, Ld, dtype, scale, out, lse, false);

@@ -40,6 +40,7 @@
 #include <cstring>
 
 #include "depth_mask.cuh"
+#include "fwd_softmax.cuh"
 #include "moda_internal.h"
 #include "sm100_ptx.cuh"
 #include "tmap_host.h"
@@ -62,20 +63,6 @@ constexpr int kMmaWarp = 9;
 constexpr int kSoftmaxRegs = 216;
 constexpr int kControlRegs = 72;
 constexpr uint32_t kNoPollLimit = 0;  // drains: time bound only
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Of every 8 column pairs of a row, pairs kPolyFrom..7 take exp2 from the
-// FMA-pipe polynomial, the rest from the MUFU unit (which alone would be
-// as busy as the tensor core at d = 128).
-#ifndef MODA_POLY_FROM
-#define MODA_POLY_FROM 8
-#endif
-constexpr int kPolyFrom = MODA_POLY_FROM;
-// P is handed to the PV MMA in this many chunks (128 / kPChunks keys each).
-#ifndef MODA_PCHUNKS
-#define MODA_PCHUNKS 1
-#endif
-constexpr int kPChunks = MODA_PCHUNKS;
-static_assert(kPChunks == 1 || kPChunks == 2 || kPChunks == 4, "P chunks");
 
 struct TcFwdParams {
     CUtensorMap tm_q, tm_k, tm_v, tm_kd, tm_vd;
@@ -97,7 +84,7 @@ struct __align__(8) Bars {
     uint64_t empty[kStages];
     uint64_t raw_full[kStages];  // 8-bit depth tile landed (before dequantisation)
     uint64_t s_full[2];
-    uint64_t p_full[2][4];  // [tile][P chunk]
+    uint64_t p_full[2];
     uint64_t o_final[2];
     uint64_t drain;
     uint32_t tmem_base;
@@ -222,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&bars->s_full[i], 1);
-            for (int c = 0; c < kPChunks; ++c) ptx::mbar_init(&bars->p_full[i][c], 4);  // one per warp
+            ptx::mbar_init(&bars->p_full[i], 4);  // one arrival per warp
             ptx::mbar_init(&bars->o_final[i], 1);
         }
         ptx::mbar_init(&bars->drain, 1);
@@ -363,25 +350,18 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                 for (int i = 0; i < 2; ++i) {
                     if (!ok) break;
                     if (part(i, x)) {
-                        // O_i += P_i V, fed chunk by chunk as the softmax
-                        // publishes P (32 keys per chunk = 2 MMA K-steps).
+                        // O_i += P_i V once the softmax has published P_i
                         const int cnt = i ? cnt_p1 : cnt_p0;
-#pragma unroll
-                        for (int c = 0; c < kPChunks; ++c) {
-                            if (!wait_all(&bars->p_full[i][c], cnt & 1)) {
-                                flag_timeout(p, bars);
-                                ok = false;
-                                break;
-                            }
-                            ptx::tc_fence_after();
-#pragma unroll
-                            for (int kk = 0; kk < 8 / kPChunks; ++kk) {
-                                const int k = (8 / kPChunks) * c + kk;
-                                ptx::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8, vd + (uint64_t)(k * 128),
-                                                 idesc_pv, (cnt > 0 || k > 0) ? 1u : 0u);
-                            }
+                        if (!wait_all(&bars->p_full[i], cnt & 1)) {
+                            flag_timeout(p, bars);
+                            ok = false;
+                            break;
                         }
-                        if (!ok) break;
+                        ptx::tc_fence_after();
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            ptx::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8, vd + (uint64_t)(k * 128),
+                                        idesc_pv, (cnt > 0 || k > 0) ? 1u : 0u);
                         if (i) ++cnt_p1; else ++cnt_p0;
                     }
                     if (next && part(i, x + 1)) {
@@ -470,108 +450,12 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                 break;
             }
             ptx::tc_fence_after();
-            float s[128];
-            {
-                uint32_t su[128];
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    ptx::tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&su[c * 32]));
-                ptx::tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(su[c]);
-            }
-            if (x < n_seq) {
-                const int kbase = x * kBN;
-                if (kbase + kBN - 1 > t) {
-#pragma unroll
-                    for (int c = 0; c < 128; ++c)
-                        if (kbase + c > t) s[c] = -INFINITY;
-                }
-            } else {
-                // same-token mask: this row's depth rows are [tl*Ld, (tl+1)*Ld)
-                // of the unit's depth range (selected slots only)
-                uint32_t vis[4];
-                depth_col_mask(tl * p.Ld - (x - n_seq) * kBN, p.Ld, has_sel, sel, vis);
-#pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (!((vis[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
-            }
-            float mx;
-            {
-                float mp[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) mp[e] = ptx::max3(s[e], s[8 + e], s[16 + e]);
-#pragma unroll
-                for (int c = 24; c < 120; c += 16)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) mp[e] = ptx::max3(mp[e], s[c + e], s[c + 8 + e]);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) mp[e] = fmaxf(mp[e], s[120 + e]);
-                mx = ptx::max3(ptx::max3(mp[0], mp[1], mp[2]), ptx::max3(mp[3], mp[4], mp[5]),
-                               fmaxf(mp[6], mp[7]));
-            }
-            const float mxs = mx * sl2;
-            if (__any_sync(0xffffffffu, mxs > m + kRescaleThreshold)) {
-                // Move the exponent reference of every row of the warp to its
-                // running max; rescale l and the O already accumulated (every
-                // earlier P V has completed: S of this item was committed
-                // after it).
-                const float mnew = fmaxf(m, mxs);
-                const float corr = (mnew == -INFINITY) ? 1.f : ptx::ex2(m - mnew);
-                if (it > 0) {
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        ptx::tmem_ld32(tO + c * 32, o);
-                        ptx::tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-                        ptx::tmem_st32(tO + c * 32, o);
-                    }
-                }
-                l *= corr;
-                m = mnew;
-            }
-            const float mref = (m == -INFINITY) ? 0.f : m;
-            const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(-mref, -mref);
-            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                             make_float2(0.f, 0.f)};
-            // P in kPChunks chunks of 32 keys: each chunk goes to TMEM and is
-            // published at once, so the PV MMA starts on it while later
-            // chunks are still being exponentiated.
-#pragma unroll
-            for (int ch = 0; ch < kPChunks; ++ch) {
-                constexpr int kPairs = 64 / kPChunks;  // packed columns per chunk
-                uint32_t pk[kPairs];
-#pragma unroll
-                for (int e = 0; e < kPairs; ++e) {
-                    const int c = ch * kPairs + e;
-                    const float2 xv = ptx::fma2(make_float2(s[2 * c], s[2 * c + 1]), sl2x2, nm2);
-                    float2 pv;
-                    if ((c & 7) >= kPolyFrom) {
-                        pv = ptx::exp2_poly2(xv);  // FMA pipe
-                    } else {
-                        pv.x = ptx::ex2(xv.x);     // MUFU
-                        pv.y = ptx::ex2(xv.y);
-                    }
-                    acc[c & 3] = ptx::add2(acc[c & 3], pv);
-                    pk[e] = ptx::pack_bf16x2(pv.x, pv.y);
-                }
-#pragma unroll
-                for (int q = 0; q < kPairs / 16; ++q)
-                    ptx::tmem_st16(tS + ch * kPairs + q * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[q * 16]));
-                ptx::tmem_wait_st();
-                ptx::tc_fence_before();
-                // one arrival per warp: 128 per-thread arrivals on one
-                // barrier word serialise on the tile's critical chain
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&bars->p_full[i][ch]);
-            }
-            {
-                const float2 a01 = ptx::add2(acc[0], acc[1]), a23 = ptx::add2(acc[2], acc[3]);
-                const float2 a = ptx::add2(a01, a23);
-                l += a.x + a.y;
-            }
+            softmax_item(tS, tO, x < n_seq, x * kBN, t, tl * p.Ld - (x - n_seq) * kBN, p.Ld, has_sel, sel, sl2,
+                         it, m, l);
+            // one arrival per warp: 128 per-thread arrivals on one barrier
+            // word serialise on the tile's critical chain
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&bars->p_full[i]);
             ++it;
         }
         if (ok) {

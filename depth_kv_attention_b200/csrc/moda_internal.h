@@ -87,6 +87,9 @@ cudaError_t launch_quantize_q8(const void* x, long long rows, int d, moda_dtype 
 // Tensor-core kernels for sm_100a (moda_fwd_sm100.cu, moda_bwd_sm100.cu).
 bool fwd_tc_supported(const FwdArgs& a);
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s);
+// The CTA-pair forward (moda_fwd_pair_sm100.cu): bf16 depth (not 8-bit).
+bool fwd_pair_supported(const FwdArgs& a);
+cudaError_t launch_fwd_pair(const FwdArgs& a, cudaStream_t s);
 bool bwd_tc_supported(const BwdArgs& a);
 cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s);
 // The forward's FMA-pipe exp2 applied element-wise (test hook).

@@ -73,8 +73,12 @@ typedef enum {
 typedef enum { MODA_BF16 = 0, MODA_F32 = 1 } moda_dtype;
 
 /* Kernel family selector for moda_fwd_ex / moda_bwd_ex.  AUTO picks the
- * tensor-core path when the shape supports it, else SIMT. */
-typedef enum { MODA_IMPL_AUTO = 0, MODA_IMPL_SIMT = 1, MODA_IMPL_TC = 2 } moda_impl;
+ * tensor-core path when the shape supports it, else SIMT. MODA_IMPL_TC2 runs
+ * the forward on CTA pairs (one M = 256 MMA drives two SMs; bf16 depth only,
+ * else MODA_ERR_UNSUPPORTED): the same results, slower than the single-CTA
+ * forward that TC and AUTO use on this hardware, kept as a selectable
+ * variant. The backward has one tensor-core form, which TC and TC2 select. */
+typedef enum { MODA_IMPL_AUTO = 0, MODA_IMPL_SIMT = 1, MODA_IMPL_TC = 2, MODA_IMPL_TC2 = 3 } moda_impl;
 
 /* Version of this ABI (MODA_ABI_VERSION of the library). */
 int moda_abi_version(void);

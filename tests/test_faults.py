@@ -17,14 +17,18 @@ moda = pytest.importorskip("depth_kv_attention_b200")
 TIMEOUT = 6  # MODA_ERR_DEVICE_TIMEOUT
 
 
-def test_bounded_wait_reports_timeout_and_context_survives():
+@pytest.mark.parametrize("impl", ["tc", "tc2"])
+def test_bounded_wait_reports_timeout_and_context_survives(impl):
+    """Both tensor-core forwards: the single-CTA kernel and the CTA-pair
+    kernel (whose expired waits also raise the peer CTA's abort flag and
+    still meet at the final cluster barrier)."""
     w = Workload("fault", 1, 640, 16, 2, 128, 5, "bf16", 41)
     x = make_inputs(w)
     xc = to_cuda(x)
     assert moda.moda_device_status() == 0
     moda.moda_debug_set_wait_limit(1)
     try:
-        moda.moda_fwd(xc["q"], xc["k"], xc["v"], xc["kd"], xc["vd"], w.scale, impl="tc")
+        moda.moda_fwd(xc["q"], xc["k"], xc["v"], xc["kd"], xc["vd"], w.scale, impl=impl)
         st = moda.moda_device_status()
     finally:
         moda.moda_debug_set_wait_limit(0)
@@ -32,7 +36,7 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     # the status word is cleared by the read
     assert moda.moda_device_status() == 0
     # the context is intact: a normal call after the expired waits is correct
-    out, lse = moda.moda_fwd(xc["q"], xc["k"], xc["v"], xc["kd"], xc["vd"], w.scale, impl="tc")
+    out, lse = moda.moda_fwd(xc["q"], xc["k"], xc["v"], xc["kd"], xc["vd"], w.scale, impl=impl)
     torch.cuda.synchronize()
     assert moda.moda_device_status() == 0
     ro, rl = oracle.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], w.scale)

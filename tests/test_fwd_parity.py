@@ -17,10 +17,11 @@ moda = pytest.importorskip("depth_kv_attention_b200")
 
 
 def impls_for(w: Workload):
-    """Kernel families a shape runs on: SIMT always, tensor cores when supported."""
+    """Kernel families a shape runs on: SIMT always; on the tensor cores the
+    CTA-pair forward ("tc") and the single-CTA forward ("tc2")."""
     out = ["simt"]
     if w.dtype == "bf16" and w.d == 128 and 128 % w.G == 0:
-        out.append("tc")
+        out += ["tc", "tc2"]
     return out
 
 
@@ -68,7 +69,7 @@ def test_tiny_f32_workload():
     check_full(WORKLOADS["tiny_f32"], "simt")
 
 
-@pytest.mark.parametrize("impl", ["simt", "tc"])
+@pytest.mark.parametrize("impl", ["simt", "tc", "tc2"])
 def test_t4k_full(impl):
     w = WORKLOADS["t4k"]
     if impl not in impls_for(w):
@@ -112,7 +113,7 @@ def test_t16k_b2_sampled_with_depth_difference(impl):
 
 def test_t64k_sampled():
     w = WORKLOADS["t64k"]
-    check_sampled(w, impls_for(w)[-1], heads=list(range(w.Hq)), n_rows=256)
+    check_sampled(w, "tc", heads=list(range(w.Hq)), n_rows=256)
 
 
 def test_packed_depth_matches_native():
