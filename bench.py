@@ -376,6 +376,45 @@ def measure_q8(moda, w, x, world, kernel, step_bf16, step_ld0, steps, warmup):
                       f"{steps} calls each"}
 
 
+def measure_write_step(moda, w, x, world, steps, warmup):
+    """The write step of one layer at this workload's shape: its key / value
+    projections (x [B*T, Hq*d] @ W [Hq*d, Hkv*d], torch GEMMs standing in
+    for the model's) written (a) to contiguous k, v and then copied into
+    depth slot 0 by moda_depth_write, or (b) straight into the slot through
+    moda_depth_slot_layout's strided views (no copy pass). Interleaved."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7)
+    dm = w.Hq * w.d
+    xin = torch.randn(w.B * w.T, dm, device="cuda", generator=g).to(torch.bfloat16)
+    wk = (torch.randn(dm, w.Hkv * w.d, device="cuda", generator=g) / dm ** 0.5).to(torch.bfloat16)
+    wv = (torch.randn(dm, w.Hkv * w.d, device="cuda", generator=g) / dm ** 0.5).to(torch.bfloat16)
+    k = torch.empty(w.B, w.T, w.Hkv, w.d, device="cuda", dtype=torch.bfloat16)
+    v = torch.empty_like(k)
+    kd, vd = x["kd"], x["vd"]
+    views = (moda.depth_slot_view(kd, 0).view(w.B * w.T, w.Hkv * w.d),
+             moda.depth_slot_view(vd, 0).view(w.B * w.T, w.Hkv * w.d))
+
+    def copy_path():
+        torch.mm(xin, wk, out=k.view(w.B * w.T, -1))
+        torch.mm(xin, wv, out=v.view(w.B * w.T, -1))
+        moda.moda_depth_write(k, v, kd, vd, 0)
+
+    def strided_path():
+        torch.mm(xin, wk, out=views[0])
+        torch.mm(xin, wv, out=views[1])
+
+    def write_only():
+        moda.moda_depth_write(k, v, kd, vd, 0)
+    ms_c, ms_s, ms_w = timed_interleaved([copy_path, strided_path, write_only], steps, warmup, world)
+    del xin, wk, wv, k, v
+    return {"proj_plus_depth_write_ms": ms_c, "proj_into_slot_ms": ms_s, "depth_write_ms": ms_w,
+            "depth_write_gbs": 4 * w.B * w.T * w.Hkv * w.d * 2 / (ms_w * 1e-3) / 1e9,
+            "saved_vs_copy": 1.0 - ms_s / ms_c,
+            "timing": f"projections of one layer (torch GEMMs, x [{w.B * w.T}, {dm}] @ [{dm}, "
+                      f"{w.Hkv * w.d}] for k and v) into contiguous k, v + moda_depth_write, or into "
+                      f"the slot views; interleaved, {steps} calls each"}
+
+
 def depth_stream_bytes(w) -> int:
     """Algorithmic bytes of the depth stream: kd and vd read once."""
     return 2 * w.B * w.T * w.Ld * w.Hkv * w.d * (2 if w.dtype == "bf16" else 4)
@@ -389,26 +428,34 @@ def depth_stream_gbs(w, ms, ms0):
     return depth_stream_bytes(w) / dt / 1e9 if dt > 0 else None
 
 
-def code_hash(path: str) -> str:
-    """SHA-256 (16 hex digits) of a CUDA source with its comments and all
+def code_hash(paths) -> str:
+    """SHA-256 (16 hex digits) of CUDA sources with their comments and all
     whitespace removed: it changes when the code changes, not when a comment
     or the layout does."""
-    with open(path) as f:
-        src = f.read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    src = re.sub(r"//[^\n]*", "", src)
-    src = re.sub(r"\s+", "", src)
-    return hashlib.sha256(src.encode()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for path in ([paths] if isinstance(paths, str) else paths):
+        with open(path) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        src = re.sub(r"\s+", "", src)
+        h.update(src.encode())
+    return h.hexdigest()[:16]
 
 
-def traffic_for(kernel_src: str):
+# The forward kernel's code: its file and the headers its device code uses.
+FWD_SOURCES = [os.path.join(ROOT, "depth_kv_attention_b200", "csrc", f)
+               for f in ("moda_fwd_sm100.cu", "fwd_softmax.cuh", "sm100_ptx.cuh", "depth_mask.cuh")]
+
+
+def traffic_for(kernel_srcs):
     """DRAM bytes per launch from the committed ncu summary, or None when the
     kernel's code changed since the counters were taken."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         t = json.load(f)
-    if t.get("code_sha256_16") != code_hash(kernel_src):
+    if t.get("code_sha256_16") != code_hash(kernel_srcs):
         return None
     return t.get("dram_bytes_per_launch")
 
@@ -576,6 +623,7 @@ def main():
             step_fwd_packed()
         ms_n, ms_p, ms_fp, ms_pf = timed_interleaved([step, step_pack, step_fwd_packed, step_pack_fwd],
                                                      args.extra_steps, args.warmup, world)
+        extra["write_step"] = measure_write_step(moda, w, x, world, args.extra_steps, args.warmup)
         extra["pack_depth"] = {
             "t_fwd_native_ms": ms_n, "t_pack_ms": ms_p, "t_fwd_packed_ms": ms_fp,
             "t_pack_plus_fwd_packed_ms": ms_pf, "pack_vs_native": ms_pf / ms_n - 1.0,
@@ -606,8 +654,8 @@ def main():
         del staging
         torch.cuda.empty_cache()
 
-    kernel_src = os.path.join(ROOT, "depth_kv_attention_b200", "csrc",
-                              "moda_simt.cu" if args.kernel == "simt" else "moda_fwd_sm100.cu")
+    kernel_src = ([os.path.join(ROOT, "depth_kv_attention_b200", "csrc", "moda_simt.cu")]
+                  if args.kernel == "simt" else FWD_SOURCES)
     peak = peaks["bf16_tflops"]
     achieved = flops_rank / (launch_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
