@@ -177,3 +177,25 @@ def test_slot_layout_is_the_native_slot():
     with pytest.raises(moda.ModaError):
         moda.moda_depth_slot_layout(2, 5, 2, 4, 3, 3)
 
+
+
+def test_header_is_plain_c_and_links():
+    """include/moda.h compiles as C99 and a C program links against
+    libmoda.so and runs the argument checks (no GPU needed)."""
+    import shutil
+    import subprocess
+    import tempfile
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = os.path.join(ROOT, "tests", "c", "abi_client.c")
+    libdir = os.path.dirname(moda.LIB_PATH)
+    with tempfile.TemporaryDirectory() as tmp:
+        exe = os.path.join(tmp, "abi_client")
+        r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), src,
+                            "-o", exe, os.path.join(libdir, "libmoda.so"), f"-Wl,-rpath,{libdir}"],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+        r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+        assert r.returncode == 0, (r.stdout, r.stderr)
+        assert r.stdout.split() == ["MODA_ERR_WORKSPACE", "0"]
