@@ -259,8 +259,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // One thread runs the MMA schedule (a single-thread tcgen05.mma issue
-        // costs about 45 cycles, a warp-wide one predicated on one lane about
-        // 80, against 64 cycles of tensor work for a 128x128x16 MMA).
+        // costs about 60 cycles, a warp-wide one predicated on one lane 80-90,
+        // against 64 cycles of tensor work for a 128x128x16 MMA; measured on
+        // the B200).
         if (lane == 0) {
             constexpr uint32_t idesc_half = ptx::idesc_bf16_f32(128, 64, 0, 0);
             constexpr uint32_t idesc_ts = ptx::idesc_bf16_f32(128, kD, 0, 1);
@@ -644,8 +645,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // One thread runs the MMA schedule (a single-thread tcgen05.mma issue
-        // costs about 45 cycles, a warp-wide one predicated on one lane about
-        // 80, against 64 cycles of tensor work for a 128x128x16 MMA).
+        // costs about 60 cycles, a warp-wide one predicated on one lane 80-90,
+        // against 64 cycles of tensor work for a 128x128x16 MMA; measured on
+        // the B200).
         if (lane == 0) {
             constexpr uint32_t idesc_ss = ptx::idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t idesc_ts = ptx::idesc_bf16_f32(128, kD, 0, 1);

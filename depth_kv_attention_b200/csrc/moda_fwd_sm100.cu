@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // One thread runs the MMA schedule: a tcgen05.mma issued by a single
-        // thread costs about 45 cycles, against about 80 when the whole warp
+        // thread costs about 60 cycles, against 80-90 when the whole warp
         // executes it predicated on one lane (measured on the B200), and the
         // tensor core finishes a 128x128x16 MMA in 64 cycles, so only the
         // single-thread form keeps it fed. Descriptors are formed once per
