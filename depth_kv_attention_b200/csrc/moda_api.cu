@@ -87,6 +87,9 @@ moda_status run_fwd(FwdArgs& a, void* stream, moda_impl impl) {
     if ((impl == MODA_IMPL_TC || impl == MODA_IMPL_TC2) && !tc_ok) return MODA_ERR_UNSUPPORTED;
     if (impl == MODA_IMPL_TC2 && !fwd_pair_supported(a)) return MODA_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // a query-token range is a tensor-core forward option only
+    if ((a.q_tok0 || a.q_tok1) && (!tc_ok || impl == MODA_IMPL_SIMT || impl == MODA_IMPL_TC2))
+        return MODA_ERR_UNSUPPORTED;
     if (impl == MODA_IMPL_SIMT || (impl == MODA_IMPL_AUTO && !tc_ok)) e = launch_fwd_simt(a, s);
     else if (impl == MODA_IMPL_TC2) e = launch_fwd_pair(a, s);
     else e = launch_fwd_tc(a, s);
@@ -370,6 +373,43 @@ size_t moda_fwd_host_staging_bytes(int B, int T, int Hq, int Hkv, int d, int Ld,
     return host_staging_layout(B, T, Hq, Hkv, d, Ld, dtype, offs);
 }
 
+namespace {
+
+// RAII holder of the extra streams and events of the pipelined host forward.
+struct HostPipe {
+    cudaStream_t sc = nullptr, so = nullptr;
+    cudaEvent_t ev[2 * 64 + 1] = {};
+    int n_ev = 0;
+    ~HostPipe() {
+        for (int i = 0; i < n_ev; ++i) cudaEventDestroy(ev[i]);  // released once recorded work completes
+        if (sc) cudaStreamDestroy(sc);
+        if (so) cudaStreamDestroy(so);
+    }
+    cudaEvent_t event() {
+        cudaEvent_t e = nullptr;
+        if (n_ev >= (int)(sizeof(ev) / sizeof(ev[0])) ||
+            cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess)
+            return nullptr;
+        ev[n_ev++] = e;
+        return e;
+    }
+};
+
+// Token rows [t0, t1) of every batch of a [B, T, row_elems] tensor, host <-> device.
+bool copy_rows(void* dst, const void* src, int B, int T, size_t row_bytes, int t0, int t1, cudaMemcpyKind kind,
+               cudaStream_t s) {
+    if (row_bytes == 0 || t1 <= t0) return true;
+    for (int b = 0; b < B; ++b) {
+        const size_t off = ((size_t)b * T + t0) * row_bytes;
+        if (cudaMemcpyAsync(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off,
+                            (size_t)(t1 - t0) * row_bytes, kind, s) != cudaSuccess)
+            return false;
+    }
+    return true;
+}
+
+}  // namespace
+
 moda_status moda_fwd_host(const void* q, const void* k, const void* v, const void* kd, const void* vd,
                           int B, int T, int Hq, int Hkv, int d, int Ld, moda_dtype dtype, float scale,
                           void* out, float* lse, void* staging, size_t staging_bytes, void* stream) {
@@ -391,22 +431,79 @@ moda_status moda_fwd_host(const void* q, const void* k, const void* v, const voi
     void* dout = base + offs[5];
     float* dlse = lse ? reinterpret_cast<float*>(base + offs[6]) : nullptr;
     const size_t esz = dtype == MODA_F32 ? 4 : 2;
-    const size_t nq = (size_t)B * T * Hq * d * esz, nkv = (size_t)B * T * Hkv * d * esz;
-    const size_t ndep = (size_t)B * T * Ld * Hkv * d * esz;
+    const size_t rq = (size_t)Hq * d * esz, rkv = (size_t)Hkv * d * esz, rdep = (size_t)Ld * Hkv * d * esz;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // inputs to the device (one cudaMemcpyAsync per tensor)
-    const void* src[5] = {q, k, v, kd, vd};
-    void* dst[5] = {dq, dk, dv, dkd, dvd};
-    const size_t nb[5] = {nq, nkv, nkv, ndep, ndep};
-    for (int i = 0; i < 5; ++i)
-        if (nb[i] && cudaMemcpyAsync(dst[i], src[i], nb[i], cudaMemcpyHostToDevice, s) != cudaSuccess)
-            return MODA_ERR_CUDA;
-    st = moda_fwd_ex(dq, dk, dv, dkd, dvd, B, T, Hq, Hkv, d, Ld, dtype, scale, dout, dlse, stream,
-                     MODA_IMPL_AUTO);
+
+    FwdArgs a;
+    st = fill_fwd(a, dq, dk, dv, dkd, dvd, B, T, Hq, Hkv, d, Ld, dtype, scale, dout, dlse, false);
     if (st != MODA_OK) return st;
-    if (cudaMemcpyAsync(out, dout, nq, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MODA_ERR_CUDA;
-    if (lse && cudaMemcpyAsync(lse, dlse, (size_t)B * Hq * T * sizeof(float), cudaMemcpyDeviceToHost, s) !=
+    const int unit = fwd_tc_supported(a) ? fwd_tc_unit_tokens(a) : 0;
+    const int nblk = unit ? (T + unit - 1) / unit : 0;
+    if (nblk < 2) {
+        // one pass: inputs to the device, the forward, outputs back
+        const void* src[5] = {q, k, v, kd, vd};
+        void* dst[5] = {dq, dk, dv, dkd, dvd};
+        const size_t rb[5] = {rq, rkv, rkv, rdep, rdep};
+        for (int i = 0; i < 5; ++i)
+            if (!copy_rows(dst[i], src[i], B, T, rb[i], 0, T, cudaMemcpyHostToDevice, s)) return MODA_ERR_CUDA;
+        st = run_fwd(a, stream, MODA_IMPL_AUTO);
+        if (st != MODA_OK) return st;
+        if (!copy_rows(out, dout, B, T, rq, 0, T, cudaMemcpyDeviceToHost, s)) return MODA_ERR_CUDA;
+        if (lse && cudaMemcpyAsync(lse, dlse, (size_t)B * Hq * T * sizeof(float), cudaMemcpyDeviceToHost, s) !=
+                       cudaSuccess)
+            return MODA_ERR_CUDA;
+        return MODA_OK;
+    }
+    // Pipelined over chunks of query tokens (whole work units): the caller's
+    // stream copies chunk j's rows of q, k, v, kd, vd; an internal stream runs
+    // the forward of chunk j's queries once they are in (causal: they need
+    // the keys of chunks 0..j only, copied before them on the same stream);
+    // a second internal stream copies chunk j's output rows back while the
+    // next chunks are copied and computed. The caller's stream waits for all
+    // of it at the end. A chunk's last key tile (128 keys) and last depth
+    // chunk (128 depth rows) reach past its last token: those keys are masked
+    // (P = 0), but 0 * NaN from a row not yet copied would still reach O, so
+    // each chunk also copies the keys up to 128 tokens and the depth rows up
+    // to 128 rows ahead (every row once: the copies continue where the last
+    // one ended).
+    HostPipe hp;
+    if (cudaStreamCreateWithFlags(&hp.sc, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&hp.so, cudaStreamNonBlocking) != cudaSuccess)
+        return MODA_ERR_CUDA;
+    const int nch = nblk < 8 ? nblk : 8;
+    const int ahead_kv = 128, ahead_dep = Ld > 0 ? (128 + Ld - 1) / Ld : 0;
+    int kv_end = 0, dep_end = 0;  // tokens copied so far of k, v and of kd, vd
+    for (int j = 0; j < nch; ++j) {
+        const int t0 = (int)((long long)nblk * j / nch) * unit;
+        const int t1 = j + 1 == nch ? T : (int)((long long)nblk * (j + 1) / nch) * unit;
+        const int kv_to = t1 + ahead_kv < T ? t1 + ahead_kv : T;
+        const int dep_to = t1 + ahead_dep < T ? t1 + ahead_dep : T;
+        if (!copy_rows(dq, q, B, T, rq, t0, t1, cudaMemcpyHostToDevice, s) ||
+            !copy_rows(dk, k, B, T, rkv, kv_end, kv_to, cudaMemcpyHostToDevice, s) ||
+            !copy_rows(dv, v, B, T, rkv, kv_end, kv_to, cudaMemcpyHostToDevice, s) ||
+            !copy_rows(dkd, kd, B, T, rdep, dep_end, dep_to, cudaMemcpyHostToDevice, s) ||
+            !copy_rows(dvd, vd, B, T, rdep, dep_end, dep_to, cudaMemcpyHostToDevice, s))
+            return MODA_ERR_CUDA;
+        kv_end = kv_to;
+        dep_end = dep_to;
+        cudaEvent_t in = hp.event(), done = hp.event();
+        if (!in || !done) return MODA_ERR_CUDA;
+        if (cudaEventRecord(in, s) != cudaSuccess || cudaStreamWaitEvent(hp.sc, in, 0) != cudaSuccess)
+            return MODA_ERR_CUDA;
+        a.q_tok0 = t0;
+        a.q_tok1 = t1;
+        st = run_fwd(a, hp.sc, MODA_IMPL_TC);
+        if (st != MODA_OK) return st;
+        if (cudaEventRecord(done, hp.sc) != cudaSuccess || cudaStreamWaitEvent(hp.so, done, 0) != cudaSuccess)
+            return MODA_ERR_CUDA;
+        if (!copy_rows(out, dout, B, T, rq, t0, t1, cudaMemcpyDeviceToHost, hp.so)) return MODA_ERR_CUDA;
+    }
+    // the so stream already waits for the last chunk's forward, hence for all
+    if (lse && cudaMemcpyAsync(lse, dlse, (size_t)B * Hq * T * sizeof(float), cudaMemcpyDeviceToHost, hp.so) !=
                    cudaSuccess)
+        return MODA_ERR_CUDA;
+    cudaEvent_t fin = hp.event();
+    if (!fin || cudaEventRecord(fin, hp.so) != cudaSuccess || cudaStreamWaitEvent(s, fin, 0) != cudaSuccess)
         return MODA_ERR_CUDA;
     return MODA_OK;
 }

@@ -69,6 +69,7 @@ struct TcFwdParams {
     void* out;
     float* lse;
     int B, T, Hq, Hkv, G, n, Ld, nblk;
+    int tb_lo, nblk_q;  // token blocks tb_lo .. tb_lo + nblk_q - 1 of each (b, kv-head) in this launch
     float sl2;  // scale * log2(e)
     int depth_packed;
     const unsigned long long* depth_sel;  // [B,T] slot masks or null
@@ -172,8 +173,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
     // first within each. CTAs in flight then share one kv-head's K/V stream
     // in L2 (at T = 64K one head's K + V is 32 MB; all four heads' streams
     // together exceed the 126 MB L2), and the lightest blocks come last.
-    const int bh = blockIdx.x / p.nblk;
-    const int tb = p.nblk - 1 - blockIdx.x % p.nblk;
+    const int bh = blockIdx.x / p.nblk_q;
+    const int tb = p.tb_lo + p.nblk_q - 1 - blockIdx.x % p.nblk_q;
     const int b = bh / p.Hkv, kvh = bh % p.Hkv;
     const int n = p.n;
     const int t0 = tb * 2 * n;
@@ -579,6 +580,12 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s) {
     p.lse = a.lse;
     p.B = a.B; p.T = a.T; p.Hq = a.Hq; p.Hkv = a.Hkv; p.G = G; p.n = n; p.Ld = a.Ld;
     p.nblk = (a.T + 2 * n - 1) / (2 * n);
+    // query-token range of this launch, in whole units of 2n tokens
+    if (a.q_tok0 % (2 * n) != 0 || a.q_tok0 < 0 || a.q_tok1 < 0 || a.q_tok1 > a.T) return cudaErrorInvalidValue;
+    p.tb_lo = a.q_tok0 / (2 * n);
+    const int tb_hi = a.q_tok1 ? (a.q_tok1 + 2 * n - 1) / (2 * n) : p.nblk;
+    p.nblk_q = tb_hi - p.tb_lo;
+    if (p.nblk_q <= 0) return cudaSuccess;
     p.sl2 = a.scale * 1.4426950408889634f;
     p.depth_packed = packed ? 1 : 0;
     p.depth_sel = a.depth_sel;
@@ -590,7 +597,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s) {
     auto kern = q8 ? moda_fwd_tc_kernel<true> : moda_fwd_tc_kernel<false>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
-    const long long grid = (long long)p.nblk * a.B * a.Hkv;
+    const long long grid = (long long)p.nblk_q * a.B * a.Hkv;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
     kern<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(p);
     return cudaGetLastError();

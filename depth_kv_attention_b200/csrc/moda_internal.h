@@ -41,6 +41,11 @@ struct FwdArgs {
     const float* vd_scale;
     unsigned int* status;     // device status word
     unsigned int wait_limit;  // bounded-wait polls (0 = kernel default)
+    // Query tokens [q_tok0, q_tok1) of this launch (tensor-core forward only;
+    // q_tok1 == 0: to T). Keys and depth rows are read from the full tensors,
+    // so the keys 0 .. q_tok1-1 must be in place; q_tok0 is a multiple of
+    // fwd_tc_unit_tokens().
+    int q_tok0, q_tok1;
 };
 
 struct BwdArgs {
@@ -86,6 +91,8 @@ cudaError_t launch_quantize_q8(const void* x, long long rows, int d, moda_dtype 
 
 // Tensor-core kernels for sm_100a (moda_fwd_sm100.cu, moda_bwd_sm100.cu).
 bool fwd_tc_supported(const FwdArgs& a);
+// Tokens per work unit of the tensor-core forward (two 128-row query tiles).
+inline int fwd_tc_unit_tokens(const FwdArgs& a) { return 2 * (128 / a.G); }
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s);
 // The CTA-pair forward (moda_fwd_pair_sm100.cu): bf16 depth (not 8-bit).
 bool fwd_pair_supported(const FwdArgs& a);

@@ -132,14 +132,30 @@ def test_packed_depth_matches_native():
     compare("packed lse", f64(l2), rl, "bf16", what="lse")
 
 
-def test_fwd_host_entry_matches_device_forward():
-    """moda_fwd_host (host buffers in and out, device staging) gives the
-    device-pointer forward's output bit for bit, and the oracle's."""
-    w = Workload("host", 2, 333, 16, 2, 128, 5, "bf16", 22)
+HOST_CASES = [
+    # G = 8: 32-token units, 8 pipelined chunks, two batches
+    Workload("host", 2, 333, 16, 2, 128, 5, "bf16", 22),
+    # G = 1: 256-token units, so a chunk's last 128-key tile and depth chunk
+    # reach into the next chunk's rows
+    Workload("host_g1", 1, 700, 4, 4, 128, 3, "bf16", 23, depth_std=4.0),
+    # one unit only: the single-pass path
+    Workload("host_one", 1, 20, 8, 1, 128, 2, "bf16", 24),
+]
+
+
+@pytest.mark.parametrize("w", HOST_CASES, ids=[w.name for w in HOST_CASES])
+def test_fwd_host_entry_matches_device_forward(w):
+    """moda_fwd_host (host buffers in and out, device staging, pipelined over
+    chunks of query tokens) gives the device-pointer forward's output bit for
+    bit, and the oracle's. The staging buffer starts as NaN: a key or depth
+    row read before its copy (even a masked one, whose P is 0) would show."""
     x = make_inputs(w)
     pinned = {k: v.pin_memory() for k, v in x.items()}
+    B, T, Hq, Hkv, d, Ld = w.B, w.T, w.Hq, w.Hkv, w.d, w.Ld
+    staging = torch.full((moda.moda_fwd_host_staging_bytes(B, T, Hq, Hkv, d, Ld, torch.bfloat16),),
+                         0xFF, dtype=torch.uint8, device="cuda")
     out_h, lse_h = moda.moda_fwd_from_host(pinned["q"], pinned["k"], pinned["v"], pinned["kd"],
-                                           pinned["vd"], w.scale)
+                                           pinned["vd"], w.scale, staging=staging)
     out, lse = run_fwd(w, x, "auto")
     assert torch.equal(out_h, out.cpu()) and torch.equal(lse_h, lse.cpu())
     ro, rl = oracle.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], w.scale)
