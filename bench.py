@@ -650,7 +650,8 @@ def main():
         e2e = {"value": flops_job / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                "api": "moda_fwd_host (C ABI): pinned host inputs -> device staging -> forward -> "
-                      "out, lse to pinned host, then a stream synchronize"}
+                      "out, lse to pinned host (copies and forward pipelined over chunks of query "
+                      "tokens), then a stream synchronize"}
         del staging
         torch.cuda.empty_cache()
 
