@@ -470,7 +470,7 @@ moda_status moda_fwd_host(const void* q, const void* k, const void* v, const voi
     if (cudaStreamCreateWithFlags(&hp.sc, cudaStreamNonBlocking) != cudaSuccess ||
         cudaStreamCreateWithFlags(&hp.so, cudaStreamNonBlocking) != cudaSuccess)
         return MODA_ERR_CUDA;
-    const int nch = nblk < 8 ? nblk : 8;
+    const int nch = nblk < 16 ? nblk : 16;
     const int ahead_kv = 128, ahead_dep = Ld > 0 ? (128 + Ld - 1) / Ld : 0;
     int kv_end = 0, dep_end = 0;  // tokens copied so far of k, v and of kd, vd
     for (int j = 0; j < nch; ++j) {

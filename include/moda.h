@@ -348,7 +348,7 @@ moda_status moda_fwd_packed(const void* q, const void* k, const void* v,
  * device-to-host copies of out and lse. No pages describe this; it is the
  * boundary a host program without device buffers of its own uses.
  * When the tensor-core forward serves the shape and T spans at least two of
- * its work units (2 * 128 / G tokens), the call pipelines up to 8 chunks of
+ * its work units (2 * 128 / G tokens), the call pipelines up to 16 chunks of
  * query tokens: the copies of chunk j run on `stream` while the forward of
  * the chunks before it runs on a stream of the library's own and their
  * outputs are copied back on another (the causal mask makes a chunk's
