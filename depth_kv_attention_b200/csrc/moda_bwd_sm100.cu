@@ -106,6 +106,7 @@ struct __align__(8) Bars {
     uint64_t full[4];            // ring slots
     uint64_t empty[4];
     uint64_t s_full, dp_full, p_full, p_full2, fin, drain, dp_read;
+    uint64_t p_ready;            // dq kernel: P of the item written (one arrival per compute warp)
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -131,6 +132,7 @@ __device__ __forceinline__ void init_bars(Bars* bars, int stages, int p_count) {
     ptx::mbar_init(&bars->fin, 1);
     ptx::mbar_init(&bars->drain, 1);
     ptx::mbar_init(&bars->dp_read, 8);
+    ptx::mbar_init(&bars->p_ready, 8);
     bars->abort_flag = 0;
     ptx::fence_barrier_init();
     ptx::fence_proxy_async_smem();
@@ -548,18 +550,19 @@ static_assert(kDqSmem <= 232448, "shared memory per CTA");
 // R[x % 2] and dP(x) in R[(x + 1) % 2]. The compute warps write P(x) and
 // dS~(x) in bf16 over S(x) (each column half: dS~ at its columns 0-31, P at
 // 32-63; for a depth item the lo term of dS~ over the half's dP columns
-// 0-31, already read). The MMA warp issues, in this order (tcgen05.mma
-// operations of one CTA execute in issue order):
+// 0-31, already read). Each compute warp publishes P(x) (p_ready) before it
+// reads dP(x). The MMA warp issues, in this order (tcgen05.mma operations of
+// one CTA execute in issue order):
 //   S(x+1) = Q K(x+1)^T   into R[(x+1) % 2], as soon as the compute warps
 //                         have loaded dP(x) from there (dp_read, before they
 //                         form dS~(x))
-//   dQ~   += dS~(x) K(x)  A = dS~(x) from R[x % 2]  \ once dS~(x) and P(x)
-//   Bq    += P(x) K(x)    A = P(x) from R[x % 2]    / are written (p_full)
+//   Bq    += P(x) K(x)    A = P(x) from R[x % 2], while dS~(x) is formed
+//   dQ~   += dS~(x) K(x)  A = dS~(x) from R[x % 2], once it is written (p_full)
 //   dP(x+1) = dO V(x+1)^T into R[x % 2], after both have read it
-// so S(x+1) runs while the compute warps form dS~(x), and the compute warps
-// exponentiate S(x+1) while dQ~, Bq and dP(x+1) run. A depth item issues
-// dQ~ += lo(x) K(x) (A from R[(x+1) % 2]) after dQ~ and Bq, and S(x+1) only
-// after that.
+// so S(x+1) and Bq run while the compute warps form dS~(x), and the compute
+// warps exponentiate S(x+1) while dQ~ and dP(x+1) run. A depth item issues
+// dQ~ += lo(x) K(x) (A from R[(x+1) % 2]) after dQ~, and S(x+1) only after
+// that.
 // Measured against two other arrangements on the wide-GQA workload (8192
 // tokens, G = 32): S(x+1) only after dS~(x) (1.23 ms) and P / dS~ in shared
 // memory with SS MMAs and dO in TMEM (1.42 ms) against 1.21 ms for this one.
@@ -682,41 +685,35 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
             if (ok) ok = issue_s(0) && issue_dp(0);
             for (int x = 0; x < n_items && ok; ++x) {
                 // the compute warps have read dP(x) from R[(x + 1) % 2], which
-                // S(x + 1) may now overwrite (depth items: after the lo MMA)
-                if (!wait_one(&bars->dp_read, x & 1)) {
+                // S(x + 1) may now overwrite (depth items: after the lo MMA);
+                // each warp published P(x) before it read dP(x), so p_ready
+                // has completed too (and cannot run a phase ahead: P(x+1)
+                // needs S(x+1), issued below)
+                if (!wait_one(&bars->dp_read, x & 1) || !wait_one(&bars->p_ready, x & 1)) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
-                if (x >= n_kv) {
-                    if (!wait_one(&bars->p_full, x & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    ptx::tc_fence_after();
-                }
                 const bool depth_item = x >= n_kv;
                 if (!depth_item && x + 1 < n_items && !issue_s(x + 1)) {
                     ok = false;
                     break;
                 }
-                if (!depth_item) {
-                    // wait p_full only now: S(x+1) went out once dP(x) was read
-                    if (!wait_one(&bars->p_full, x & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    ptx::tc_fence_after();
-                }
                 const int sk = 2 * x;
                 const uint64_t km = mndesc(aRing + (sk % kDqStages) * kTile);
-#pragma unroll
-                for (int k = 0; k < kBK / 16; ++k)
-                    ptx::mma_ts(tmem + 256, tmem + (x & 1) * 128 + acol(k), km + mnoff(k), idesc_ts,
-                                     (x > 0 || k > 0) ? 1u : 0u);
+                // Bq += P(x) K(x) while the compute warps form dS~(x)
 #pragma unroll
                 for (int k = 0; k < kBK / 16; ++k)
                     ptx::mma_ts(tmem + 384, tmem + (x & 1) * 128 + 32 + acol(k), km + mnoff(k), idesc_ts,
+                                     (x > 0 || k > 0) ? 1u : 0u);
+                if (!wait_one(&bars->p_full, x & 1)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < kBK / 16; ++k)
+                    ptx::mma_ts(tmem + 256, tmem + (x & 1) * 128 + acol(k), km + mnoff(k), idesc_ts,
                                      (x > 0 || k > 0) ? 1u : 0u);
                 if (depth_item) {
                     // the lo term of dS~(x), then S(x + 1) over it
@@ -825,6 +822,11 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
                     for (int e = 0; e < 16; ++e) pp[e] = ptx::pack_bf16x2(pr[32 * c + 2 * e], pr[32 * c + 2 * e + 1]);
                     ptx::tmem_st16(rS + 64 * hs + 32 + 16 * c, pp);
                 }
+                // P is in TMEM: Bq += P K may go out before dS~ is formed
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&bars->p_ready);
             }
             if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->dp_full, x & 1, p.wait_limit, abort_flag))) {
                 flag_timeout(p.status, bars);
