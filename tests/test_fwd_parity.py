@@ -140,6 +140,10 @@ HOST_CASES = [
     Workload("host_g1", 1, 700, 4, 4, 128, 3, "bf16", 23, depth_std=4.0),
     # one unit only: the single-pass path
     Workload("host_one", 1, 20, 8, 1, 128, 2, "bf16", 24),
+    # no depth keys: pipelined, no kd / vd copies
+    Workload("host_ld0", 1, 300, 16, 2, 128, 0, "bf16", 25),
+    # fp32: the SIMT kernels, single pass
+    Workload("host_f32", 2, 45, 4, 2, 64, 3, "f32", 26),
 ]
 
 
@@ -152,12 +156,12 @@ def test_fwd_host_entry_matches_device_forward(w):
     x = make_inputs(w)
     pinned = {k: v.pin_memory() for k, v in x.items()}
     B, T, Hq, Hkv, d, Ld = w.B, w.T, w.Hq, w.Hkv, w.d, w.Ld
-    staging = torch.full((moda.moda_fwd_host_staging_bytes(B, T, Hq, Hkv, d, Ld, torch.bfloat16),),
+    staging = torch.full((moda.moda_fwd_host_staging_bytes(B, T, Hq, Hkv, d, Ld, pinned["q"].dtype),),
                          0xFF, dtype=torch.uint8, device="cuda")
     out_h, lse_h = moda.moda_fwd_from_host(pinned["q"], pinned["k"], pinned["v"], pinned["kd"],
                                            pinned["vd"], w.scale, staging=staging)
     out, lse = run_fwd(w, x, "auto")
     assert torch.equal(out_h, out.cpu()) and torch.equal(lse_h, lse.cpu())
     ro, rl = oracle.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], w.scale)
-    compare("host out", f64(out_h), ro, "bf16")
-    compare("host lse", f64(lse_h), rl, "bf16", what="lse")
+    compare("host out", f64(out_h), ro, w.dtype)
+    compare("host lse", f64(lse_h), rl, w.dtype, what="lse")
