@@ -194,11 +194,16 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
     // the depth chunks that overlap its own tokens' depth rows.
     // (selects rather than indexing, so that a runtime tile index keeps the
     // arrays in registers)
+    // Depth chunks [dlo_i, dhi_i) (as item indices) overlap tile i's rows
+    // i*n*Ld .. (i*n + nv_i)*Ld.
+    int dlo[2], dhi[2];
+    for (int i = 0; i < 2; ++i) {
+        const int row0 = i * n * p.Ld, row1 = row0 + nv[i] * p.Ld;
+        dlo[i] = n_seq + row0 / kBN;
+        dhi[i] = nv[i] > 0 ? n_seq + (row1 + kBN - 1) / kBN : dlo[i];
+    }
     auto part = [&](int i, int x) {
-        const int nkv_i = i ? n_kv[1] : n_kv[0], nv_i = i ? nv[1] : nv[0];
-        if (x < n_seq) return x < nkv_i;
-        const int lo = (x - n_seq) * kBN, row0 = i * n * p.Ld;
-        return nv_i > 0 && lo < row0 + nv_i * p.Ld && lo + kBN > row0;
+        return x < (i ? n_kv[1] : n_kv[0]) || (x >= (i ? dlo[1] : dlo[0]) && x < (i ? dhi[1] : dhi[0]));
     };
 
     if (threadIdx.x == 0) {
@@ -309,6 +314,11 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
             const uint32_t sRa = ptx::smem_u32(sRing);
             uint64_t dq_desc[2];
             for (int i = 0; i < 2; ++i) dq_desc[i] = ptx::umma_desc_sw128(sQa + i * kTileBytes, 16, 1024);
+            // ring slot st's K / V descriptors: the stage's offset added to the
+            // 14-bit address field of slot 0's (addresses stay below 2^18 B)
+            const uint64_t k0 = ptx::umma_desc_sw128(sRa, 16, 1024);
+            const uint64_t v0 = ptx::umma_desc_sw128(sRa, kHalfBytes, 1024);
+            constexpr uint64_t kSlotUnits = kTileBytes >> 4;
             // (a plain bounded wait: one thread, no warp vote)
             auto wait_all = [&](uint64_t* bar, uint32_t parity) {
                 return ptx::mbar_wait(bar, parity, wait_limit, abort_flag);
@@ -317,10 +327,19 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
             if (!ok) flag_timeout(p, bars);
             ptx::tc_fence_after();
             int cnt_p0 = 0, cnt_p1 = 0;
-            // S_i = Q_i K^T for the K tile in ring slot `seq`
-#define MODA_ISSUE_S(I, SEQ)                                                                   \
+            // ring position of the V tile of item x (2x + 1) and of the K tile of
+            // item x + 1 (2x + 2) as (stage, phase), advanced without divisions
+            int st_v = 1, ph_v = 0;
+            auto advance = [](int& st, int& ph) {
+                if (++st == kStages) {
+                    st = 0;
+                    ph ^= 1;
+                }
+            };
+            // S_i = Q_i K^T for the K tile in ring stage ST
+#define MODA_ISSUE_S(I, ST)                                                                    \
     do {                                                                                       \
-        const uint64_t kd_ = ptx::umma_desc_sw128(sRa + ((SEQ) % kStages) * kTileBytes, 16, 1024); \
+        const uint64_t kd_ = k0 + (uint64_t)(ST) * kSlotUnits;                                 \
         const uint64_t qd_ = dq_desc[I];                                                       \
         _Pragma("unroll") for (int k = 0; k < kD / 16; ++k) {                                  \
             const uint64_t off = (uint64_t)((k >> 2) * (kHalfBytes >> 4) + (k & 3) * 2);        \
@@ -337,15 +356,16 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                 ptx::mma_commit(&bars->empty[0]);
             }
             for (int x = 0; x < n_items && ok; ++x) {
-                const int sv = 2 * x + 1, sk = 2 * x + 2;
+                int st_k = st_v, ph_k = ph_v;
+                advance(st_k, ph_k);
                 const bool next = x + 1 < n_items;
-                ok = wait_all(&bars->full[sv % kStages], (sv / kStages) & 1);
+                ok = wait_all(&bars->full[st_v], ph_v);
                 if (!ok) {
                     flag_timeout(p, bars);
                     break;
                 }
                 ptx::tc_fence_after();
-                const uint64_t vd = ptx::umma_desc_sw128(sRa + (sv % kStages) * kTileBytes, kHalfBytes, 1024);
+                const uint64_t vd = v0 + (uint64_t)st_v * kSlotUnits;
                 bool k_ready = false;
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
@@ -367,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                     }
                     if (next && part(i, x + 1)) {
                         if (!k_ready) {
-                            if (!wait_all(&bars->full[sk % kStages], (sk / kStages) & 1)) {
+                            if (!wait_all(&bars->full[st_k], ph_k)) {
                                 flag_timeout(p, bars);
                                 ok = false;
                                 break;
@@ -375,12 +395,15 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_tc_kernel(const __grid_c
                             ptx::tc_fence_after();
                             k_ready = true;
                         }
-                        MODA_ISSUE_S(i, sk);
+                        MODA_ISSUE_S(i, st_k);
                     }
                 }
                 if (!ok) break;
-                ptx::mma_commit(&bars->empty[sv % kStages]);
-                if (next) ptx::mma_commit(&bars->empty[sk % kStages]);
+                ptx::mma_commit(&bars->empty[st_v]);
+                if (next) ptx::mma_commit(&bars->empty[st_k]);
+                st_v = st_k;
+                ph_v = ph_k;
+                advance(st_v, ph_v);
             }
 #undef MODA_ISSUE_S
             if (ok) {
