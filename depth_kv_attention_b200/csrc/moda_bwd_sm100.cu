@@ -34,6 +34,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <type_traits>
 
 #include "depth_mask.cuh"
 #include "moda_internal.h"
@@ -399,36 +400,43 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
                 hi_r = 128;
             }
             const uint32_t tH = tmem + lane_off + 128 * hs;  // this half's S^T | dP^T
+            // every query row of this half visible to every key of the warp:
+            // the loop without the per-element range test (warp-uniform)
+            const bool all_vis = __all_sync(0xffffffffu, lo_r <= 64 * hs && hi_r >= 64 * hs + 64);
+            auto tile = [&](auto masked) {
 #pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-                uint32_t sr[32], dr[32];
-                ptx::tmem_ld32(tH + 32 * c, sr);
-                ptx::tmem_ld32(tH + 64 + 32 * c, dr);
-                ptx::tmem_wait_ld();
-                uint32_t pp[16], dd[16];
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t sr[32], dr[32];
+                    ptx::tmem_ld32(tH + 32 * c, sr);
+                    ptx::tmem_ld32(tH + 64 + 32 * c, dr);
+                    ptx::tmem_wait_ld();
+                    uint32_t pp[16], dd[16];
 #pragma unroll
-                for (int e2 = 0; e2 < 16; ++e2) {
-                    float pv[2], dv[2];
-                    const int r0 = 64 * hs + 32 * c + 2 * e2;  // query row of the tile
-                    const float2 ex = exp2_pair(make_float2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -st_lse[r0]),
-                                                            fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -st_lse[r0 + 1])),
-                                                e2);
+                    for (int e2 = 0; e2 < 16; ++e2) {
+                        float pv[2], dv[2];
+                        const int r0 = 64 * hs + 32 * c + 2 * e2;  // query row of the tile
+                        const float2 ex = exp2_pair(make_float2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -st_lse[r0]),
+                                                                fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -st_lse[r0 + 1])),
+                                                    e2);
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int rr = r0 + u;
-                        float pr = u ? ex.y : ex.x;
-                        if (rr < lo_r || rr >= hi_r) pr = 0.f;
-                        pv[u] = pr;
-                        dv[u] = pr * (__uint_as_float(dr[2 * e2 + u]) - st_D[rr]);
+                        for (int u = 0; u < 2; ++u) {
+                            const int rr = r0 + u;
+                            float pr = u ? ex.y : ex.x;
+                            if (decltype(masked)::value && (rr < lo_r || rr >= hi_r)) pr = 0.f;
+                            pv[u] = pr;
+                            dv[u] = pr * (__uint_as_float(dr[2 * e2 + u]) - st_D[rr]);
+                        }
+                        pp[e2] = ptx::pack_bf16x2(pv[0], pv[1]);
+                        dd[e2] = ptx::pack_bf16x2(dv[0], dv[1]);
                     }
-                    pp[e2] = ptx::pack_bf16x2(pv[0], pv[1]);
-                    dd[e2] = ptx::pack_bf16x2(dv[0], dv[1]);
+                    // chunk c's packed columns [16c, 16c+16) lie in columns
+                    // this thread has already read
+                    ptx::tmem_st16(tH + 16 * c, pp);
+                    ptx::tmem_st16(tH + 64 + 16 * c, dd);
                 }
-                // chunk c's packed columns [16c, 16c+16) lie in columns
-                // this thread has already read
-                ptx::tmem_st16(tH + 16 * c, pp);
-                ptx::tmem_st16(tH + 64 + 16 * c, dd);
-            }
+            };
+            if (all_vis) tile(std::false_type{});
+            else tile(std::true_type{});
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             ptx::mbar_arrive(hs ? &bars->p_full2 : &bars->p_full);
@@ -800,19 +808,33 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
                 for (int c = 0; c < 2; ++c)
                     ptx::tmem_ld32(rS + 64 * hs + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&su[c * 32]));
                 ptx::tmem_wait_ld();
-                uint32_t vis[4];  // visible columns of this row
-                if (x < n_kv)
-                    depth_col_mask(0, t - x * kBK + 1, false, 0ull, vis);  // keys <= t
-                else  // the row's own depth rows (selected slots)
-                    depth_col_mask(tt * p.Ld - (x - n_kv) * kBK, p.Ld, has_sel, sel, vis);
-                const uint32_t vw[2] = {hs ? vis[2] : vis[0], hs ? vis[3] : vis[1]};
+                // a key tile wholly at or before every row of the warp needs no
+                // mask (warp-uniform test; x < n_kv is the same for the warp)
+                const bool all_vis = x < n_kv && __all_sync(0xffffffffu, x * kBK + 64 * hs + 63 <= t);
+                if (all_vis) {
 #pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const float2 e = exp2_pair(make_float2(fmaf(__uint_as_float(su[c]), sl2, -lse2),
-                                                           fmaf(__uint_as_float(su[c + 1]), sl2, -lse2)),
-                                               c / 2);
-                    pr[c] = ((vw[c >> 5] >> (c & 31)) & 1u) ? e.x : 0.f;
-                    pr[c + 1] = ((vw[c >> 5] >> ((c + 1) & 31)) & 1u) ? e.y : 0.f;
+                    for (int c = 0; c < 64; c += 2) {
+                        const float2 e = exp2_pair(make_float2(fmaf(__uint_as_float(su[c]), sl2, -lse2),
+                                                               fmaf(__uint_as_float(su[c + 1]), sl2, -lse2)),
+                                                   c / 2);
+                        pr[c] = e.x;
+                        pr[c + 1] = e.y;
+                    }
+                } else {
+                    uint32_t vis[4];  // visible columns of this row
+                    if (x < n_kv)
+                        depth_col_mask(0, t - x * kBK + 1, false, 0ull, vis);  // keys <= t
+                    else  // the row's own depth rows (selected slots)
+                        depth_col_mask(tt * p.Ld - (x - n_kv) * kBK, p.Ld, has_sel, sel, vis);
+                    const uint32_t vw[2] = {hs ? vis[2] : vis[0], hs ? vis[3] : vis[1]};
+#pragma unroll
+                    for (int c = 0; c < 64; c += 2) {
+                        const float2 e = exp2_pair(make_float2(fmaf(__uint_as_float(su[c]), sl2, -lse2),
+                                                               fmaf(__uint_as_float(su[c + 1]), sl2, -lse2)),
+                                                   c / 2);
+                        pr[c] = ((vw[c >> 5] >> (c & 31)) & 1u) ? e.x : 0.f;
+                        pr[c + 1] = ((vw[c >> 5] >> ((c + 1) & 31)) & 1u) ? e.y : 0.f;
+                    }
                 }
                 // P in bf16 over this half's S columns 32-63 (already read)
 #pragma unroll
