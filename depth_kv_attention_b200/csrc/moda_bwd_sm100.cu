@@ -865,24 +865,31 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&bars->dp_read);
+            // dS~ in bf16 (hi), and for a depth item also the lo term (two loop
+            // versions: the lo arithmetic only where it is stored)
+            auto ds_pass = [&](auto with_lo) {
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const uint32_t* dr = drr + 32 * c;
-                uint32_t dd[16], dl[16];
+                for (int c = 0; c < 2; ++c) {
+                    const uint32_t* dr = drr + 32 * c;
+                    uint32_t dd[16], dl[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float d0 = pr[32 * c + 2 * e] * (__uint_as_float(dr[2 * e]) - Drow);
-                    const float d1 = pr[32 * c + 2 * e + 1] * (__uint_as_float(dr[2 * e + 1]) - Drow);
-                    delta += d0 + d1;
-                    dd[e] = ptx::pack_bf16x2(d0, d1);
-                    // lo term: the part of dS~ the bf16 hi term drops
-                    dl[e] = ptx::pack_bf16x2(d0 - __uint_as_float(dd[e] << 16),
-                                             d1 - __uint_as_float(dd[e] & 0xffff0000u));
+                    for (int e = 0; e < 16; ++e) {
+                        const float d0 = pr[32 * c + 2 * e] * (__uint_as_float(dr[2 * e]) - Drow);
+                        const float d1 = pr[32 * c + 2 * e + 1] * (__uint_as_float(dr[2 * e + 1]) - Drow);
+                        delta += d0 + d1;
+                        dd[e] = ptx::pack_bf16x2(d0, d1);
+                        // lo term: the part of dS~ the bf16 hi term drops
+                        if (decltype(with_lo)::value)
+                            dl[e] = ptx::pack_bf16x2(d0 - __uint_as_float(dd[e] << 16),
+                                                     d1 - __uint_as_float(dd[e] & 0xffff0000u));
+                    }
+                    ptx::tmem_st16(rS + 64 * hs + 16 * c, dd);  // over this half's S(x), already read
+                    // over this half's dP(x) columns 16c.., read in chunk 0
+                    if (decltype(with_lo)::value) ptx::tmem_st16(rP + 64 * hs + 16 * c, dl);
                 }
-                ptx::tmem_st16(rS + 64 * hs + 16 * c, dd);  // over this half's S(x), already read
-                // over this half's dP(x) columns 16c.., read in chunk 0
-                if (depth_item) ptx::tmem_st16(rP + 64 * hs + 16 * c, dl);
-            }
+            };
+            if (depth_item) ds_pass(std::true_type{});
+            else ds_pass(std::false_type{});
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars->p_full);
