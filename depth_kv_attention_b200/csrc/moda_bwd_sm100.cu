@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
     uint8_t* sK = smem;
     uint8_t* sV = smem + kTile;
     uint8_t* sRing = smem + 2 * kTile;  // stage s: Q at +2s*kTile, dO at +(2s+1)*kTile
-    float* sStat = reinterpret_cast<float*>(sRing + kDkvStages * 2 * kTile);  // [lse2 | D] of the query tile
+    float* sStat = reinterpret_cast<float*>(sRing + kDkvStages * 2 * kTile);  // [-lse2 | -D] of the query tile
     Bars* bars = reinterpret_cast<Bars*>(sStat + 256);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -376,8 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
             float* st_D = sStat + 128;
             half_sync(hs);  // this half's readers of the previous tile are done
             if (r < 64) {
-                st_lse[64 * hs + r] = nl2;
-                st_D[64 * hs + r] = nD;
+                st_lse[64 * hs + r] = -nl2;  // stored negated: the packed FMA / ADD below add them
+                st_D[64 * hs + r] = -nD;
                 if (i + 1 < nq) load_stat(i + 1, nl2, nD);
             }
             const bool got = ptx::mbar_wait(hs ? &bars->dp_full : &bars->s_full, i & 1, p.wait_limit, abort_flag);
@@ -413,21 +413,21 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
                     uint32_t pp[16], dd[16];
 #pragma unroll
                     for (int e2 = 0; e2 < 16; ++e2) {
-                        float pv[2], dv[2];
                         const int r0 = 64 * hs + 32 * c + 2 * e2;  // query row of the tile
-                        const float2 ex = exp2_pair(make_float2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -st_lse[r0]),
-                                                                fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -st_lse[r0 + 1])),
-                                                    e2);
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int rr = r0 + u;
-                            float pr = u ? ex.y : ex.x;
-                            if (decltype(masked)::value && (rr < lo_r || rr >= hi_r)) pr = 0.f;
-                            pv[u] = pr;
-                            dv[u] = pr * (__uint_as_float(dr[2 * e2 + u]) - st_D[rr]);
+                        const float2 nl = *reinterpret_cast<const float2*>(st_lse + r0);
+                        const float2 nd = *reinterpret_cast<const float2*>(st_D + r0);
+                        float2 pv = exp2_pair(ptx::fma2(make_float2(__uint_as_float(sr[2 * e2]),
+                                                                    __uint_as_float(sr[2 * e2 + 1])),
+                                                        make_float2(sl2, sl2), nl),
+                                              e2);
+                        if (decltype(masked)::value) {
+                            if (r0 < lo_r || r0 >= hi_r) pv.x = 0.f;
+                            if (r0 + 1 < lo_r || r0 + 1 >= hi_r) pv.y = 0.f;
                         }
-                        pp[e2] = ptx::pack_bf16x2(pv[0], pv[1]);
-                        dd[e2] = ptx::pack_bf16x2(dv[0], dv[1]);
+                        const float2 dv = ptx::mul2(
+                            pv, ptx::add2(make_float2(__uint_as_float(dr[2 * e2]), __uint_as_float(dr[2 * e2 + 1])), nd));
+                        pp[e2] = ptx::pack_bf16x2(pv.x, pv.y);
+                        dd[e2] = ptx::pack_bf16x2(dv.x, dv.y);
                     }
                     // chunk c's packed columns [16c, 16c+16) lie in columns
                     // this thread has already read
@@ -812,11 +812,12 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
                 // mask (warp-uniform test; x < n_kv is the same for the warp)
                 const bool all_vis = x < n_kv && __all_sync(0xffffffffu, x * kBK + 64 * hs + 63 <= t);
                 if (all_vis) {
+                    const float2 sl2x2 = make_float2(sl2, sl2), nl2x2 = make_float2(-lse2, -lse2);
 #pragma unroll
                     for (int c = 0; c < 64; c += 2) {
-                        const float2 e = exp2_pair(make_float2(fmaf(__uint_as_float(su[c]), sl2, -lse2),
-                                                               fmaf(__uint_as_float(su[c + 1]), sl2, -lse2)),
-                                                   c / 2);
+                        const float2 e = exp2_pair(
+                            ptx::fma2(make_float2(__uint_as_float(su[c]), __uint_as_float(su[c + 1])), sl2x2, nl2x2),
+                            c / 2);
                         pr[c] = e.x;
                         pr[c + 1] = e.y;
                     }
@@ -866,7 +867,10 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&bars->dp_read);
             // dS~ in bf16 (hi), and for a depth item also the lo term (two loop
-            // versions: the lo arithmetic only where it is stored)
+            // versions: the lo arithmetic only where it is stored); packed fp32
+            // pairs, the row sum of dS~ in two lanes
+            const float2 nDrow = make_float2(-Drow, -Drow);
+            float2 dsum = make_float2(0.f, 0.f);
             auto ds_pass = [&](auto with_lo) {
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
@@ -874,9 +878,11 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
                     uint32_t dd[16], dl[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float d0 = pr[32 * c + 2 * e] * (__uint_as_float(dr[2 * e]) - Drow);
-                        const float d1 = pr[32 * c + 2 * e + 1] * (__uint_as_float(dr[2 * e + 1]) - Drow);
-                        delta += d0 + d1;
+                        const float2 d = ptx::mul2(
+                            make_float2(pr[32 * c + 2 * e], pr[32 * c + 2 * e + 1]),
+                            ptx::add2(make_float2(__uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1])), nDrow));
+                        dsum = ptx::add2(dsum, d);
+                        const float d0 = d.x, d1 = d.y;
                         dd[e] = ptx::pack_bf16x2(d0, d1);
                         // lo term: the part of dS~ the bf16 hi term drops
                         if (decltype(with_lo)::value)
@@ -890,6 +896,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
             };
             if (depth_item) ds_pass(std::true_type{});
             else ds_pass(std::false_type{});
+            delta += dsum.x + dsum.y;
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars->p_full);
