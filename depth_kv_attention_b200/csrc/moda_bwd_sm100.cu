@@ -117,9 +117,9 @@ __device__ __forceinline__ void flag_timeout(unsigned int* status, Bars* bars) {
     atomicOr(status, 1u);
 }
 
-// p_count: arrivals that publish P (the dQ kernel: all 256 compute threads
-// on p_full; the dK/dV kernel: each 128-thread half on its own p_full /
-// p_full2).
+// p_count: arrivals that publish P, one per compute warp (the dQ kernel: 8 on
+// p_full; the dK/dV kernel: each 4-warp half on its own p_full / p_full2).
+// Per-thread arrivals on one barrier word would serialise on the chain.
 __device__ __forceinline__ void init_bars(Bars* bars, int stages, int p_count) {
     ptx::mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < stages; ++s) {
@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
         nq = (c_hi - t_first + n - 1) / n;
     }
 
-    if (threadIdx.x == 0) init_bars(bars, kDkvStages, kComputeThreads / 2);
+    if (threadIdx.x == 0) init_bars(bars, kDkvStages, kComputeThreads / 64);
     if (warp == 0) {
         ptx::tmem_alloc(&bars->tmem_base, 512);
         ptx::tmem_relinquish();
@@ -439,7 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
             else tile(std::true_type{});
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
-            ptx::mbar_arrive(hs ? &bars->p_full2 : &bars->p_full);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(hs ? &bars->p_full2 : &bars->p_full);
         }
         if (ok) {
             const bool got = ptx::mbar_wait(&bars->fin, 0, p.wait_limit, abort_flag);
@@ -595,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
     const int n_dep = (nv * p.Ld + kBK - 1) / kBK;
     const int n_items = n_kv + n_dep;
 
-    if (threadIdx.x == 0) init_bars(bars, kDqStages, kComputeThreads);
+    if (threadIdx.x == 0) init_bars(bars, kDqStages, kComputeThreads / 32);
     if (warp == 0) {
         ptx::tmem_alloc(&bars->tmem_base, 512);
         ptx::tmem_relinquish();
@@ -899,7 +900,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dq_kernel(const __grid_c
             delta += dsum.x + dsum.y;
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
-            ptx::mbar_arrive(&bars->p_full);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&bars->p_full);
         }
         if (ok && !__all_sync(0xffffffffu, ptx::mbar_wait(&bars->fin, 0, p.wait_limit, abort_flag))) {
             flag_timeout(p.status, bars);
