@@ -395,17 +395,17 @@ struct HostPipe {
     }
 };
 
-// Token rows [t0, t1) of every batch of a [B, T, row_elems] tensor, host <-> device.
+// Token rows [t0, t1) of every batch of a [B, T, row_bytes] tensor, host <-> device:
+// one 2D copy (B rows of (t1 - t0) * row_bytes, pitch T * row_bytes), or a
+// plain copy when the range is the whole tensor.
 bool copy_rows(void* dst, const void* src, int B, int T, size_t row_bytes, int t0, int t1, cudaMemcpyKind kind,
                cudaStream_t s) {
     if (row_bytes == 0 || t1 <= t0) return true;
-    for (int b = 0; b < B; ++b) {
-        const size_t off = ((size_t)b * T + t0) * row_bytes;
-        if (cudaMemcpyAsync(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off,
-                            (size_t)(t1 - t0) * row_bytes, kind, s) != cudaSuccess)
-            return false;
-    }
-    return true;
+    const size_t off = (size_t)t0 * row_bytes, width = (size_t)(t1 - t0) * row_bytes, pitch = (size_t)T * row_bytes;
+    char* d = static_cast<char*>(dst) + off;
+    const char* h = static_cast<const char*>(src) + off;
+    if (B == 1 || width == pitch) return cudaMemcpyAsync(d, h, width * B, kind, s) == cudaSuccess;
+    return cudaMemcpy2DAsync(d, pitch, h, pitch, width, (size_t)B, kind, s) == cudaSuccess;
 }
 
 }  // namespace
