@@ -14,12 +14,13 @@
 //      from the stored output, sees all keys of its rows, and so also forms
 //      the exact D = D~ + sum_j P_j (dP_j - D~) and corrects dq for D - D~;
 //      dq accumulates in TMEM and is written once, in bf16
-//   2. dk, dv: KV-major tensor-core kernel (reads the exact D); partial sums
-//      of a key tile over a chunk of query tiles go to fp32 accumulators
-//      with vector reductions
-//   3. dkd, dvd: the same kernel with 128-row depth chunks as the key tiles
-//      and a same-token mask (each depth row owned by one CTA, bf16 stores)
-//   4. dk, dv = bf16(accumulators)
+//   2. one launch of the KV-major tensor-core kernel (reads the exact D):
+//      dk, dv CTAs first (partial sums of a key tile over a chunk of query
+//      tiles go to fp32 accumulators with vector reductions), then dkd, dvd
+//      CTAs (128-row depth chunks as the key tiles, a same-token mask, each
+//      depth row owned by one CTA, bf16 stores), which fill the SMs the
+//      last wave of dk, dv CTAs leaves idle
+//   3. dk, dv = bf16(accumulators)
 // Splitting dq from dk/dv recomputes S and dP once more but removes the
 // per-pair fp32 dq reductions, which for wide GQA (G = 32, 4 tokens per
 // 128-row tile) would move gigabytes through L2.
@@ -141,16 +142,21 @@ __device__ __forceinline__ void init_bars(Bars* bars, int stages, int p_count) {
 
 // ===================================================================== dk, dv
 struct DkvParams {
-    CUtensorMap tm_q, tm_do, tm_k, tm_v;  // in depth mode tm_k / tm_v map kd / vd
+    CUtensorMap tm_q, tm_do, tm_k, tm_v, tm_kd, tm_vd;
     const float* lse;
     const float* rowD;
     float* dk_acc;  // sequence mode: [B,T,Hkv,d] fp32, zeroed before the launch
     float* dv_acc;
     void* dkd;      // depth mode: [B,T,Ld,Hkv,d] bf16 outputs
     void* dvd;
-    int depth_mode, Ld;
+    int Ld;
     const unsigned long long* depth_sel;  // depth mode: [B,T] slot masks or null
     int B, T, Hq, Hkv, G, n, gshift, qchunk;
+    // grid: n_seq_ctas sequence-mode CTAs (key tile fastest, then chunk of
+    // query tokens, then (b, kv-head)), then n_dep_chunks depth-mode CTAs per
+    // (b, kv-head) (depth chunk fastest)
+    int nkt, n_chunks, n_dep_chunks;
+    long long n_seq_ctas;
     float sl2, scale;
     unsigned int* status;
     unsigned int wait_limit;
@@ -160,14 +166,16 @@ constexpr int kDkvSmem = 2 * kTile + kDkvStages * 2 * kTile + 2 * 128 * 4 + 256 
 static_assert(kDkvSmem <= 232448, "shared memory per CTA");
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
-// Sequence mode: one CTA per (key tile = blockIdx.x, chunk of query tokens =
-// blockIdx.y, (b, kv-head) = blockIdx.z), causal mask, partial sums reduced
-// into fp32 accumulators.
-// Depth mode (the depth keys' gradients dkd, dvd): the "key tile" is the
-// 128-row depth chunk blockIdx.x of the [B, T*Ld, Hkv, d] view, the query
-// tiles are those holding the chunk's tokens, the mask keeps each depth row
-// to its own token's G heads, and since one CTA owns every row of its chunk
-// the results are written directly in bf16.
+// One launch holds both kinds of CTA: the sequence-mode CTAs first, then the
+// depth-mode ones, which are short and fill the SMs that the last wave of
+// long sequence-mode CTAs leaves idle.
+// Sequence mode: one CTA per (key tile, chunk of query tokens, (b, kv-head)),
+// causal mask, partial sums reduced into fp32 accumulators.
+// Depth mode (the depth keys' gradients dkd, dvd): the "key tile" is a
+// 128-row depth chunk of the [B, T*Ld, Hkv, d] view, the query tiles are
+// those holding the chunk's tokens, the mask keeps each depth row to its own
+// token's G heads, and since one CTA owns every row of its chunk the results
+// are written directly in bf16.
 // Each 128-row query tile is processed as two halves of 64 query rows that
 // ping-pong like the forward's two query tiles: while the compute warps of
 // one half form P^T and dS^T, the tensor core runs the other half's MMAs.
@@ -190,11 +198,27 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     volatile int* abort_flag = &bars->abort_flag;
-    const int b = blockIdx.z / p.Hkv, kvh = blockIdx.z % p.Hkv;
-    const int j0 = blockIdx.x * kBK;  // first key row (sequence) or depth row (depth mode)
+    // (key tile or depth chunk, chunk of query tokens, (b, kv-head)) of this CTA
+    const bool depth_mode = (long long)blockIdx.x >= p.n_seq_ctas;
+    int bx, by, bz;
+    if (!depth_mode) {
+        const int r = (int)blockIdx.x / p.nkt;
+        bx = (int)blockIdx.x % p.nkt;
+        by = r % p.n_chunks;
+        bz = r / p.n_chunks;
+    } else {
+        const long long r = (long long)blockIdx.x - p.n_seq_ctas;
+        bx = (int)(r % p.n_dep_chunks);
+        by = 0;
+        bz = (int)(r / p.n_dep_chunks);
+    }
+    const CUtensorMap* tm_kx = depth_mode ? &p.tm_kd : &p.tm_k;
+    const CUtensorMap* tm_vx = depth_mode ? &p.tm_vd : &p.tm_v;
+    const int b = bz / p.Hkv, kvh = bz % p.Hkv;
+    const int j0 = bx * kBK;  // first key row (sequence) or depth row (depth mode)
     const int n = p.n;
     int t_first, nq;
-    if (p.depth_mode) {
+    if (depth_mode) {
         // tokens whose depth rows meet [j0, j0 + 128), whole query tiles
         const int last_row = min(j0 + kBK, p.T * p.Ld) - 1;
         t_first = (j0 / p.Ld) / n * n;
@@ -203,8 +227,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
         // A chunk is qchunk query tiles of absolute tokens [c*qchunk*n, ...);
         // the CTAs in flight at once cover one or two chunks. Key tiles that
         // no row of the chunk can see exit at once.
-        const int c_lo = blockIdx.y * p.qchunk * n;
-        const int c_hi = min(p.T, (blockIdx.y + 1) * p.qchunk * n);
+        const int c_lo = by * p.qchunk * n;
+        const int c_hi = min(p.T, (by + 1) * p.qchunk * n);
         t_first = max(j0, c_lo);  // a multiple of n
         if (t_first >= c_hi) return;
         nq = (c_hi - t_first + n - 1) / n;
@@ -231,13 +255,13 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
         if (lead) {
             ptx::prefetch_tmap(&p.tm_q);
             ptx::prefetch_tmap(&p.tm_do);
-            ptx::prefetch_tmap(&p.tm_k);
-            ptx::prefetch_tmap(&p.tm_v);
+            ptx::prefetch_tmap(tm_kx);
+            ptx::prefetch_tmap(tm_vx);
         }
         ptx::mbar_arrive_expect_tx_lead(&bars->kv_full, 2 * kTile, lead);
         for (int hf = 0; hf < 2; ++hf) {
-            ptx::tma_load_4d_lead(sK + hf * kHalf, &p.tm_k, &bars->kv_full, hf * 64, kvh, j0, b, lead);
-            ptx::tma_load_4d_lead(sV + hf * kHalf, &p.tm_v, &bars->kv_full, hf * 64, kvh, j0, b, lead);
+            ptx::tma_load_4d_lead(sK + hf * kHalf, tm_kx, &bars->kv_full, hf * 64, kvh, j0, b, lead);
+            ptx::tma_load_4d_lead(sV + hf * kHalf, tm_vx, &bars->kv_full, hf * 64, kvh, j0, b, lead);
         }
         int issued = 0;
         for (int i = 0; i < nq; ++i) {
@@ -348,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
         const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
         const int j = j0 + r;            // this thread's key
         // depth mode: is depth row j (slot j % Ld of token j / Ld) selected?
-        const bool j_selected = !p.depth_mode || !p.depth_sel || j >= p.T * p.Ld ||
+        const bool j_selected = !depth_mode || !p.depth_sel || j >= p.T * p.Ld ||
                                 ((p.depth_sel[(long long)b * p.T + j / p.Ld] >> (j % p.Ld)) & 1ull);
         const float sl2 = p.sl2;
         const int gshift = p.gshift;
@@ -391,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
             // is seen by rows of tokens tq0 + (rr >> gshift) >= j; depth mode,
             // depth row j is seen only by the rows of its own token j / Ld.
             int lo_r, hi_r;
-            if (p.depth_mode) {
+            if (depth_mode) {
                 const int td = j < p.T * p.Ld ? j / p.Ld : -1;
                 lo_r = (td - tq0) * p.G;
                 hi_r = (td < 0 || !j_selected) ? lo_r : lo_r + p.G;
@@ -450,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_bwd_dkdv_kernel(const __grid
             }
         }
         ptx::tc_fence_after();
-        if (ok && p.depth_mode) {
+        if (ok && depth_mode) {
             // dkd (scaled) and dvd of this chunk's depth rows, written directly
             const bool valid = j < p.T * p.Ld;
             const long long off = (((long long)b * p.T * p.Ld + (valid ? j : 0)) * p.Hkv + kvh) * kD;
@@ -1038,7 +1062,7 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s) {
     // ---- dk, dv
     DkvParams pk;
     memset(&pk, 0, sizeof(pk));
-    pk.tm_q = tm_q; pk.tm_do = tm_do; pk.tm_k = tm_k; pk.tm_v = tm_v;
+    pk.tm_q = tm_q; pk.tm_do = tm_do; pk.tm_k = tm_k; pk.tm_v = tm_v; pk.tm_kd = tm_kd; pk.tm_vd = tm_vd;
     pk.lse = f.lse; pk.rowD = a.rowD; pk.dk_acc = a.dk_acc; pk.dv_acc = a.dv_acc;
     pk.B = f.B; pk.T = f.T; pk.Hq = f.Hq; pk.Hkv = f.Hkv; pk.G = G; pk.n = n; pk.gshift = gshift;
     pk.sl2 = f.scale * kLog2e; pk.scale = f.scale;
@@ -1058,25 +1082,25 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s) {
     if ((e = cudaFuncSetAttribute(moda_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDkvSmem)) !=
         cudaSuccess)
         return e;
-    const int n_chunks = ((f.T + n - 1) / n + pk.qchunk - 1) / pk.qchunk;
-    moda_bwd_dkdv_kernel<<<dim3(nkt, n_chunks, f.B * f.Hkv), kThreads, kDkvSmem, s>>>(pk);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-    // ---- dkd, dvd: the same kernel over the depth chunks
+    // sequence-mode CTAs (key tile, chunk of query tokens, (b, kv-head)), then
+    // with depth keys the depth-mode CTAs (128-row depth chunk, (b, kv-head))
+    pk.nkt = nkt;
+    pk.n_chunks = ((f.T + n - 1) / n + pk.qchunk - 1) / pk.qchunk;
+    pk.n_seq_ctas = (long long)nkt * pk.n_chunks * f.B * f.Hkv;
+    long long grid_kv = pk.n_seq_ctas;
     if (f.Ld > 0) {
-        DkvParams pd = pk;
-        pd.tm_k = tm_kd;
-        pd.tm_v = tm_vd;
-        pd.depth_mode = 1;
-        pd.Ld = f.Ld;
-        pd.depth_sel = f.depth_sel;
-        pd.dkd = a.dkd;
-        pd.dvd = a.dvd;
         const long long chunks = ((long long)f.T * f.Ld + kBK - 1) / kBK;
         if (chunks > 0x7fffffffLL) return cudaErrorInvalidValue;
-        moda_bwd_dkdv_kernel<<<dim3((unsigned)chunks, 1, f.B * f.Hkv), kThreads, kDkvSmem, s>>>(pd);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        pk.n_dep_chunks = (int)chunks;
+        pk.Ld = f.Ld;
+        pk.depth_sel = f.depth_sel;
+        pk.dkd = a.dkd;
+        pk.dvd = a.dvd;
+        grid_kv += chunks * f.B * f.Hkv;
     }
+    if (grid_kv > 0x7fffffffLL) return cudaErrorInvalidValue;
+    moda_bwd_dkdv_kernel<<<(unsigned)grid_kv, kThreads, kDkvSmem, s>>>(pk);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     // ---- dk, dv to bf16
     const long long n4 = (long long)f.B * f.T * f.Hkv * kD / 4;
