@@ -312,9 +312,10 @@ def make_step(moda, w, x, mode, kernel, depth_sel=None):
                       impl=kernel)
         moda.moda_bwd(x["q"], x["k"], x["v"], x["kd"], x["vd"], out, lse, x["dout"], w.scale,
                       grads=grads, workspace=ws, impl=kernel)
-    # forward 1; tensor-core backward: dq, dk/dv, depth dk/dv (Ld > 0), 2
-    # conversions; SIMT backward: D~, dq, dk/dv, depth (Ld > 0)
-    bwd = (3 if kernel == "simt" else 4) + (1 if w.Ld else 0)
+    # forward 1; tensor-core backward: dq, one dk/dv launch (its grid also
+    # holds the depth dk/dv CTAs), 2 conversions; SIMT backward: D~, dq,
+    # dk/dv, depth (Ld > 0)
+    bwd = 3 + (1 if w.Ld else 0) if kernel == "simt" else 4
     return step, 1 + bwd, out, lse
 
 
