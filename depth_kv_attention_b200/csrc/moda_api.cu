@@ -470,6 +470,21 @@ moda_status moda_fwd_host(const void* q, const void* k, const void* v, const voi
     if (cudaStreamCreateWithFlags(&hp.sc, cudaStreamNonBlocking) != cudaSuccess ||
         cudaStreamCreateWithFlags(&hp.so, cudaStreamNonBlocking) != cudaSuccess)
         return MODA_ERR_CUDA;
+    // An error after work went onto the internal streams still orders the
+    // caller's stream after that work (or, if that cannot be enqueued, waits
+    // for it here), so the caller may release its buffers once its own stream
+    // is done.
+    auto fail = [&](moda_status e) {
+        cudaStream_t inner[2] = {hp.sc, hp.so};
+        for (cudaStream_t t : inner) {
+            cudaEvent_t j = nullptr;
+            const bool joined = cudaEventCreateWithFlags(&j, cudaEventDisableTiming) == cudaSuccess &&
+                                cudaEventRecord(j, t) == cudaSuccess && cudaStreamWaitEvent(s, j, 0) == cudaSuccess;
+            if (j) cudaEventDestroy(j);
+            if (!joined) cudaStreamSynchronize(t);
+        }
+        return e;
+    };
     const int nch = nblk < 16 ? nblk : 16;
     const int ahead_kv = 128, ahead_dep = Ld > 0 ? (128 + Ld - 1) / Ld : 0;
     int kv_end = 0, dep_end = 0;  // tokens copied so far of k, v and of kd, vd
@@ -483,28 +498,28 @@ moda_status moda_fwd_host(const void* q, const void* k, const void* v, const voi
             !copy_rows(dv, v, B, T, rkv, kv_end, kv_to, cudaMemcpyHostToDevice, s) ||
             !copy_rows(dkd, kd, B, T, rdep, dep_end, dep_to, cudaMemcpyHostToDevice, s) ||
             !copy_rows(dvd, vd, B, T, rdep, dep_end, dep_to, cudaMemcpyHostToDevice, s))
-            return MODA_ERR_CUDA;
+            return fail(MODA_ERR_CUDA);
         kv_end = kv_to;
         dep_end = dep_to;
         cudaEvent_t in = hp.event(), done = hp.event();
-        if (!in || !done) return MODA_ERR_CUDA;
+        if (!in || !done) return fail(MODA_ERR_CUDA);
         if (cudaEventRecord(in, s) != cudaSuccess || cudaStreamWaitEvent(hp.sc, in, 0) != cudaSuccess)
-            return MODA_ERR_CUDA;
+            return fail(MODA_ERR_CUDA);
         a.q_tok0 = t0;
         a.q_tok1 = t1;
         st = run_fwd(a, hp.sc, MODA_IMPL_TC);
-        if (st != MODA_OK) return st;
+        if (st != MODA_OK) return fail(st);
         if (cudaEventRecord(done, hp.sc) != cudaSuccess || cudaStreamWaitEvent(hp.so, done, 0) != cudaSuccess)
-            return MODA_ERR_CUDA;
-        if (!copy_rows(out, dout, B, T, rq, t0, t1, cudaMemcpyDeviceToHost, hp.so)) return MODA_ERR_CUDA;
+            return fail(MODA_ERR_CUDA);
+        if (!copy_rows(out, dout, B, T, rq, t0, t1, cudaMemcpyDeviceToHost, hp.so)) return fail(MODA_ERR_CUDA);
     }
     // the so stream already waits for the last chunk's forward, hence for all
     if (lse && cudaMemcpyAsync(lse, dlse, (size_t)B * Hq * T * sizeof(float), cudaMemcpyDeviceToHost, hp.so) !=
                    cudaSuccess)
-        return MODA_ERR_CUDA;
+        return fail(MODA_ERR_CUDA);
     cudaEvent_t fin = hp.event();
     if (!fin || cudaEventRecord(fin, hp.so) != cudaSuccess || cudaStreamWaitEvent(s, fin, 0) != cudaSuccess)
-        return MODA_ERR_CUDA;
+        return fail(MODA_ERR_CUDA);
     return MODA_OK;
 }
 

@@ -366,7 +366,10 @@ moda_status moda_fwd_packed(const void* q, const void* k, const void* v,
  * lse hold the results when the stream reaches the end of the call (e.g.
  * after moda_device_status(stream)). Errors: as moda_fwd, MODA_ERR_WORKSPACE
  * for a missing or short staging buffer, MODA_ERR_CUDA if a copy cannot be
- * enqueued.
+ * enqueued. After an error that comes once copies or launches are enqueued,
+ * `stream` is still ordered after all of them (else the call waits for them
+ * before it returns), so the buffers may be released once `stream` is done;
+ * out and lse are then undefined.
  */
 size_t moda_fwd_host_staging_bytes(int B, int T, int Hq, int Hkv, int d, int Ld,
                                    moda_dtype dtype);
