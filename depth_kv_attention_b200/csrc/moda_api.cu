@@ -1,7 +1,8 @@
 // Host side of the C ABI declared in include/moda.h: argument validation,
-// kernel-family selection and launch. No allocation, no synchronisation
-// (except moda_device_status), no state beyond the device status word and
-// the test hook's wait limit.
+// kernel-family selection and launch. No device allocation and no
+// synchronisation (except moda_device_status, and moda_fwd_host's own
+// streams and events), no state beyond the device status word and the test
+// hook's wait limit.
 #include <atomic>
 #include <cstdint>
 #include <cstring>

@@ -20,9 +20,12 @@
  *
  * Conventions shared by every entry point
  *   - Every tensor argument is a DEVICE pointer to a dense, row-major tensor in
- *     the layout stated below, aligned to 16 bytes. The caller owns every
- *     buffer; the library never allocates, frees or synchronises (except in
- *     moda_device_status) and keeps no per-call state.
+ *     the layout stated below, aligned to 16 bytes (moda_fwd_host: host
+ *     buffers, see there). The caller owns every buffer; the library never
+ *     allocates device memory, frees or synchronises (except in
+ *     moda_device_status, and in moda_fwd_host, which creates two streams and
+ *     its events for the call and, after an error, may wait for them) and
+ *     keeps no per-call state.
  *   - Layouts:  q, out, dout, dq   [B, T, Hq, d]
  *               k, v, dk, dv       [B, T, Hkv, d]
  *               kd, vd, dkd, dvd   [B, T, Ld, Hkv, d]   (depth keys/values of a
